@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of the sharded mixed-precision Adam step (ZeRO) on B200.
+
+One step = one ``zero_step`` call through the C ABI: the reduce-scatter of Nd gradient
+replicas, the fp16/bf16 unscale and overflow check, Adam/AdamW on every rank's fp32 shard,
+and the bf16 all-gather to the Nd weight replicas, all Nd simulated ranks in this GPU's memory.
+
+Default workload: ZeRO-1 on N = 124,439,808 parameters (GPT-2 small), Nd = 8 simulated ranks,
+bf16 gradients ~N(0,1e-3), AdamW (lr 6e-4, wd 0.01).  Inputs are synthetic, generated on the
+device by the seeded generator before the timed region (distinct gradients per step, cycling
+through as many sets as fit a memory budget); every step reads more than the 126 MB L2.
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent replica of the
+workload on its own GPU (the simulated ranks are already inside one GPU; there is no data-path
+collective), so per-GPU work is fixed (weak scaling) and the value is the sum over GPUs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "params updated/s and achieved HBM GB/s (% of B200 peak) per ZeRO step"
+
+# name -> workload.  bytes_per_param: algorithmic HBM traffic of one step per parameter.
+WORKLOADS = {
+    "zero1-gpt2-small": dict(
+        desc="ZeRO-1 flat N=124,439,808 (GPT-2 small), Nd=8, bf16 grads ~N(0,1e-3), AdamW "
+             "lr 6e-4 wd 0.01, bf16 weights all-gathered to 8 replicas",
+        stage=1, Nd=8, N=124_439_808, bucket=0, gdt="bf16", sigma=1e-3, kind="normal",
+        hp=dict(lr=6e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
+    "zero2-2p28-nd8": dict(
+        desc="ZeRO-2 flat N=2^28, Nd=8, bf16 grads ~N(0,1e-3), AdamW lr 1e-3 wd 0.01",
+        stage=2, Nd=8, N=1 << 28, bucket=0, gdt="bf16", sigma=1e-3, kind="normal",
+        hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
+    "zero2-1m-nd4": dict(
+        desc="ZeRO-2 N=1,000,003 (padded to ceil(N/4)), Nd=4, bf16 grads ~N(0,1e-3), Adam lr 1e-3",
+        stage=2, Nd=4, N=1_000_003, bucket=0, gdt="bf16", sigma=1e-3, kind="normal",
+        hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, loss_scale=1.0)),
+    "zero2-fp16-bucketed": dict(
+        desc="ZeRO-2 N=1.3e9 in 25M-element buckets, Nd=16, fp16 grads ~N(0,1e-4)*1024 "
+             "(loss scale 1024), AdamW lr 1e-3 wd 0.01",
+        stage=2, Nd=16, N=1_300_000_000, bucket=25_000_000, gdt="fp16", sigma=1e-4 * 1024,
+        kind="normal",
+        hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1024.0)),
+    "zero2-wide-fanin-nd64": dict(
+        desc="ZeRO-2 flat N=2^28, Nd=64, bf16 grads ~N(0,1e-3) with 1% x1e3, AdamW step 1000 "
+             "with m,v prefilled",
+        stage=2, Nd=64, N=1 << 28, bucket=0, gdt="bf16", sigma=1e-3, kind="heavy", t0=999,
+        hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
+}
+DEFAULT = "zero1-gpt2-small"
+
+
+def bytes_per_param(w) -> int:
+    # fused step: Nd 2-byte gradient reads, fp32 master/m/v read + write, Nd 2-byte weight writes
+    return 2 * w["Nd"] + 24 + 2 * w["Nd"]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_record():
+    """ncu DRAM bytes per launch of the fused kernel, valid only for the kernel source it was
+    captured from (profiles/traffic.json records that source's sha256)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "zero_sharded_optimizer_03_b200", "csrc", "zero_kernels.cuh")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if rec.get("kernels_sha256") != sha:
+        return None
+    return rec
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-i", self.gpu_id, "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU baseline
+
+def cpu_baseline(w, target_s=10.0, steps=None):
+    """Time the CPU oracle (single thread, as it stands) on a bounded sample of the workload:
+    the first n parameters, n sized for about target_s seconds of oracle work."""
+    import numpy as np
+
+    import oracle
+    import synth
+    Nd = w["Nd"]
+    odt = oracle.FP16 if w["gdt"] == "fp16" else oracle.BF16
+    sdt = synth.FP16 if w["gdt"] == "fp16" else synth.BF16
+
+    def make(n):
+        grads = [synth.fill_host(synth.NORMAL, sdt, synth.SEED, synth.grad_stream(1, r), n,
+                                 sigma=w["sigma"]) for r in range(Nd)]
+        S, Np, _ = oracle.partition(n, Nd)
+        p = np.zeros(Np, np.float32)
+        p[:n] = synth.fill_host(synth.NORMAL, synth.F32, synth.SEED, synth.MASTER_STREAM, n,
+                                sigma=0.02)
+        return grads, p, np.zeros(Np, np.float32), np.zeros(Np, np.float32), [
+            np.zeros(n, np.uint16) for _ in range(Nd)]
+
+    n0 = 1 << 18
+    g, p, m, v, reps = make(n0)
+    t = time.perf_counter()
+    oracle.zero12_step(Nd, n0, 0, odt, g, p, m, v, reps, w["hp"], 0)
+    rate0 = n0 / (time.perf_counter() - t)
+    n = int(min(w["N"], max(n0, rate0 * target_s)))
+    g, p, m, v, reps = make(n)
+    times = []
+    tcount = 0
+    for _ in range(steps or 1):
+        t0 = time.perf_counter()
+        tcount, _, _ = oracle.zero12_step(Nd, n, w.get("bucket", 0), odt, g, p, m, v, reps,
+                                          w["hp"], tcount)
+        times.append(time.perf_counter() - t0)
+    return n, times
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--grad-sets-gb", type=float, default=24.0,
+                    help="device memory budget for distinct per-step gradient sets")
+    ap.add_argument("--n-override", type=int, default=0,
+                    help="run the workload at a different N (small cases for profiling)")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    w = dict(WORKLOADS[args.workload])
+    if args.n_override:
+        w["N"] = args.n_override
+        w["desc"] += " [N overridden to %d]" % args.n_override
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    config = {"workload": w["desc"], "N": w["N"], "Nd": w["Nd"], "stage": w["stage"],
+              "bucket": w["bucket"], "grad_dtype": w["gdt"], "state_dtype": "f32",
+              "weights_dtype": "bf16", "parallelism": "replicas (%d simulated ranks per GPU)"
+              % w["Nd"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
+              % (2 * w["Nd"] * w["N"] / 1e9)}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        n, times = cpu_baseline(w, target_s=3.0, steps=args.warmup + args.steps)
+        timed = times[args.warmup:]
+        ms = 1e3 * sum(timed) / len(timed)
+        val = n / (ms / 1e3)
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "params/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": val, "unit": "params/s", "cores": 1, "kind": "oracle",
+                                 "sample": "first %d of %d parameters, Nd=%d, one step each"
+                                 % (n, w["N"], w["Nd"])},
+                "e2e": {"value": val, "unit": "params/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import synth
+    import zero_sharded_optimizer_03_b200 as zero
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    s = torch.cuda.current_stream()
+    sp = s.cuda_stream
+
+    Nd, N, stage = w["Nd"], w["N"], w["stage"]
+    gdt = zero.ZERO_FP16 if w["gdt"] == "fp16" else zero.ZERO_BF16
+    sdt = synth.FP16 if w["gdt"] == "fp16" else synth.BF16
+    kind = synth.HEAVY if w["kind"] == "heavy" else synth.NORMAL
+    tail = float(__import__("numpy").float32(w["sigma"] * 1e3))
+    hp = zero.hparams(**w["hp"])
+    buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt)
+    synth.fill_device(buf.master[0].data_ptr(), synth.NORMAL, synth.F32, synth.SEED,
+                      synth.MASTER_STREAM, N, 0.02, cuda_stream=sp)
+    if w.get("t0"):
+        synth.fill_device(buf.exp_avg[0].data_ptr(), synth.ABS, synth.F32, synth.SEED,
+                          synth.M_STREAM, N, 1e-3, cuda_stream=sp)
+        synth.fill_device(buf.exp_avg_sq[0].data_ptr(), synth.SQUARE, synth.F32, synth.SEED,
+                          synth.V_STREAM, N, 1e-6, cuda_stream=sp)
+    buf.init_workspace(w.get("t0", 0))
+    buf.sync_params_from_master()
+
+    # distinct gradient sets (set 0 lives in buf.grads)
+    set_bytes = 2 * Nd * N
+    nsets = int(max(1, min(args.warmup + args.steps, args.grad_sets_gb * 1e9 // set_bytes)))
+    gsets = [buf.grads] + [[torch.empty(N, dtype=buf.grads[0].dtype, device=dev)
+                            for _ in range(Nd)] for _ in range(nsets - 1)]
+    states = []
+    for k, gs in enumerate(gsets):
+        for r in range(Nd):
+            synth.fill_device(gs[r].data_ptr(), kind, sdt, synth.SEED,
+                              synth.grad_stream(k + 1, r), N, w["sigma"], tail, cuda_stream=sp)
+        st = zero.zero_state_t.from_buffer_copy(buf.state)
+        for r in range(Nd):
+            st.grads[r] = gs[r].data_ptr()
+        states.append(st)
+    nb = 1 if w["bucket"] == 0 else -(-N // w["bucket"])
+    launches_per_step = nb + 1  # fused kernel per bucket + the overflow-repair check
+
+    def step(k, ev=None):
+        if ev is not None:
+            zero.zero_profile_events(ev[0].cuda_event, ev[1].cuda_event)
+        zero.zero_step(stage, Nd, N, w["bucket"], states[k % nsets], hp, sp)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in kev:  # create the underlying CUDA events before handing them to the library
+        a.record(s)
+        b.record(s)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    gpu_id = getattr(torch.cuda.get_device_properties(dev), "uuid", None)
+    sampler = ClockSampler(("GPU-" + str(gpu_id)) if gpu_id else str(local))
+    sampler.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record(s)
+    for k in range(args.steps):
+        step(args.warmup + k, kev[k])
+    t_stop.record(s)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms_total = t_start.elapsed_time(t_stop)
+    kern_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
+    res = buf.result()
+    assert res["overflow"] == 0 and res["skipped"] == 0, res
+
+    if dist:
+        t = torch.tensor([ms_total, kern_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, kern_ms = float(t[0]), float(t[1])
+    ms_step = ms_total / args.steps
+    value = world * N / (ms_step / 1e3)
+    bpp = bytes_per_param(w)
+    achieved = bpp * N / (kern_ms / 1e3) / 1e9
+    peak, peak_src = peaks()
+    tr = traffic_record()
+    traffic = None
+    if tr and tr.get("workload") == args.workload:
+        traffic = tr["dram_bytes_per_launch"]
+
+    # end to end through the public API: pinned host gradients -> device, step, result -> host
+    e2e = None
+    if not args.no_e2e:
+        host = [torch.empty(N, dtype=buf.grads[0].dtype, pin_memory=True) for _ in range(Nd)]
+        for r in range(Nd):
+            host[r].copy_(buf.grads[r])
+        torch.cuda.synchronize()
+        res_bytes = 48  # the workspace header zero_read_result copies back
+        e_start = torch.cuda.Event(enable_timing=True)
+        e_stop = torch.cuda.Event(enable_timing=True)
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e_start.record(s)
+        for k in range(args.e2e_steps):
+            for r in range(Nd):
+                buf.grads[r].copy_(host[r], non_blocking=True)
+            zero.zero_step(stage, Nd, N, w["bucket"], buf.state, hp, sp)
+            zero.zero_read_result(buf.ws.data_ptr(), sp)
+        e_stop.record(s)
+        torch.cuda.synchronize()
+        e_ms = e_start.elapsed_time(e_stop)
+        if dist:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        e2e = {"value": world * N / (e_ms / args.e2e_steps / 1e3), "unit": "params/s",
+               "h2d_bytes_per_step": 2 * Nd * N, "d2h_bytes_per_step": res_bytes,
+               "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, times = cpu_baseline(w)
+        cpu = {"value": n / times[0], "unit": "params/s", "cores": 1, "kind": "oracle",
+               "sample": "first %d of %d parameters, Nd=%d, one ZeRO step (%.1f s)"
+               % (n, N, Nd, times[0])}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic", "config": config,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
+                             "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                             "peak_source": peak_src, "kernel": "fused_step_kernel",
+                             "bytes_per_param": bpp, "kernel_ms": kern_ms,
+                             "frac_of_8TBs": achieved / 8000.0},
+                "hbm_gbs_per_step": bpp * N / (ms_step / 1e3) / 1e9,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+                "gpu_launches": launches_per_step * args.steps,
+                "grad_sets": nsets}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

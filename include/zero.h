@@ -1,0 +1,250 @@
+/*
+ * zero.h -- C ABI of the B200 sharded mixed-precision Adam step (ZeRO stages 1, 2 and 3).
+ *
+ * The library (libzero.so, built from zero_sharded_optimizer_03_b200/csrc) implements the
+ * data-parallel hot path of the Zero Redundancy Optimizer as described by
+ *   [P1] "ZeRO 优化器的三个阶段深度对比：显存节省与通信开销的量化分析" (wmrh.cn/news/520095)
+ *   [P2] "ZeRO 优化器：把显存“分”着用" (5688vip.com course note 03)
+ *   [P3] "ZeRO Optimization（零冗余优化）" (ai-master.cc glossary)
+ * with its collectives simulated over Nd virtual ranks whose buffers all live in the memory
+ * of one GPU: the reduce-scatter is an Nd-way fan-in read and the all-gather an Nd-way
+ * fan-out write, inside the same kernels as the optimizer arithmetic.
+ *
+ * Conventions (every entry point):
+ *   - Returns ZERO_OK (0) or a negative error code; zero_last_error() then returns a message
+ *     (thread-local, valid until the next call on the same thread).  Nothing aborts.
+ *   - The caller owns all memory.  The library never allocates device or host memory.  Device
+ *     pointers are plain CUDA device addresses (e.g. torch tensor data_ptr()).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Device
+ *     work is enqueued on it and runs asynchronously; only zero_read_result synchronizes.
+ *   - Element indices are global positions in the flat parameter vector of N elements.  The
+ *     fp32 optimizer state (master weights, exp_avg, exp_avg_sq) is stored flat and padded:
+ *     Nd*S floats with S = ceil(N/Nd); rank r's shard is the view [r*S, (r+1)*S) and elements
+ *     N .. Nd*S-1 are padding that the caller zero-fills once and the library never writes.
+ *   - 16-bit values (gradients, bf16 weights) are passed as raw uint16_t bit patterns.
+ *   - Pointers that are 16-byte aligned take the vectorised path; any other alignment is
+ *     accepted and handled element by element (same results, slower).
+ *   - An overflow (inf/NaN in the reduced gradient) is not an error: the step is skipped and
+ *     reported through the workspace (see zero_read_result).
+ *   - Numerics: each update is the element-wise rule written out in zero_adam_shard, one
+ *     fp32 round-to-nearest operation at a time, no fused multiply-add; gradient replicas are
+ *     summed in rank order 0..Nd-1.  Results do not depend on the launch configuration,
+ *     except the last bits of the reported sum of squares (fixed order for a given GPU).
+ */
+#ifndef ZERO_H
+#define ZERO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ codes and limits */
+
+#define ZERO_OK 0
+#define ZERO_EINVAL (-1) /* an argument is out of range or NULL; the message names it */
+#define ZERO_ECUDA (-2)  /* a CUDA runtime call or a kernel launch failed */
+
+#define ZERO_MAX_ND 64   /* largest number of simulated data-parallel ranks */
+
+/* gradient replica element types */
+#define ZERO_BF16 0
+#define ZERO_FP16 1
+
+/* zero_step flags */
+#define ZERO_FUSED 0     /* stages 1/2: one fused pass (default); state copies ping-pong */
+#define ZERO_TWO_PASS 1  /* stages 1/2: reduce-scatter into grad_shard, then Adam + all-gather */
+
+/* zero_allgather gates */
+#define ZERO_GATE_ALWAYS 0      /* always cast and write */
+#define ZERO_GATE_NO_OVERFLOW 1 /* write nothing if the current step has overflowed so far */
+
+/* ------------------------------------------------------------------ types */
+
+/* Partition of N elements over Nd ranks ([P1] §二: each rank keeps 1/Nd of the optimizer
+ * state; [P3] core operations: each process keeps only its own shard). */
+typedef struct {
+    int64_t N;      /* elements */
+    int32_t Nd;     /* ranks */
+    int32_t reserved;
+    int64_t S;      /* shard length ceil(N/Nd); rank r owns [r*S, min((r+1)*S, N)) */
+    int64_t Np;     /* padded length Nd*S */
+    int64_t pad;    /* Np - N */
+} zero_partition_t;
+
+/* Hyperparameters of one step.  lr may change from call to call (schedules). */
+typedef struct {
+    double lr;
+    double beta1, beta2;
+    double eps;
+    double weight_decay;  /* decoupled (AdamW); 0 gives Adam */
+    double loss_scale;    /* static fp16 loss scale the gradients carry; 1 if none */
+    int32_t grad_average; /* nonzero: g = sum/(Nd*loss_scale) (data-parallel mean); 0: sum/loss_scale */
+    int32_t reserved;
+} zero_hparams_t;
+
+/* Host copy of the step bookkeeping kept in the workspace. */
+typedef struct {
+    int64_t step;       /* completed (not skipped) updates t */
+    int64_t skipped;    /* steps skipped because of an overflow */
+    int32_t overflow;   /* 1 if the last finished step was skipped */
+    int32_t live;       /* ZERO_FUSED: index (0/1) of the state copy that holds the current state */
+    double grad_sumsq;  /* sum of squares of the last finished step's reduced gradient */
+    int32_t pending_overflow; /* overflow accumulated by the step in progress */
+    int32_t reserved;
+    double pending_sumsq;     /* sum of squares accumulated by the step in progress */
+} zero_step_result_t;
+
+/* Buffers of a whole step (zero_step).  All pointers are device pointers owned by the caller.
+ * Unused fields may be NULL. */
+typedef struct {
+    int32_t grad_dtype;  /* ZERO_BF16 or ZERO_FP16 */
+    int32_t flags;       /* ZERO_FUSED or ZERO_TWO_PASS (stages 1/2) */
+    /* stages 1/2: rank r's gradient replica (N elements) and bf16 weight replica (N elements).
+     * stage 3: rank r's gradient buffer and gathered-weight buffer for the layer being
+     * processed; layer l uses grads[r] + l*grad_layer_stride and params[r] + l*param_layer_stride
+     * (a stride of 0 reuses one layer-sized buffer, which is how a backward pass frees them). */
+    const uint16_t *grads[ZERO_MAX_ND];
+    uint16_t *params[ZERO_MAX_ND];
+    /* fp32 state, each padded (stages 1/2: Nd*S floats; stage 3: the padded layers back to back).
+     * ZERO_FUSED reads copy `live` and writes copy 1-live, so both copies must be allocated and
+     * zero-initialised in their padding; the other paths use copy 0 in place. */
+    float *master[2];
+    float *exp_avg[2];
+    float *exp_avg_sq[2];
+    float *grad_shard;      /* fp32 reduced gradient, same padded length (ZERO_TWO_PASS, stage 3) */
+    uint16_t *param_shard;  /* stage 3: bf16 weights, the Nd shards of every layer (padded) */
+    int64_t grad_layer_stride;
+    int64_t param_layer_stride;
+    void *workspace;        /* zero_workspace_bytes() bytes, initialised by zero_workspace_init */
+} zero_state_t;
+
+/* Per-GPU model-state memory in GiB (2^30 bytes). */
+typedef struct {
+    double optimizer_states, gradients, parameters, total;
+} zero_mem_t;
+
+/* ------------------------------------------------------------------ bookkeeping */
+
+/* Message of the last failed call on this thread ("" if none).  Never NULL. */
+const char *zero_last_error(void);
+
+/* Library version string, e.g. "zero-b200 1.0 sm_100a". */
+const char *zero_version(void);
+
+/* Fills *out with the partition of N elements over Nd ranks.  N >= 0 (N = 0 gives S = 0),
+ * 1 <= Nd <= ZERO_MAX_ND.  Host only. */
+int zero_partition(int64_t N, int Nd, zero_partition_t *out);
+
+/* Bytes of device workspace a step needs (a small constant: step counter, overflow flag,
+ * sum of squares, per-CTA partials).  One workspace per optimizer (it carries the step count). */
+size_t zero_workspace_bytes(void);
+
+/* Sets the workspace to "t completed updates, nothing pending, state copy 0 live".  Async. */
+int zero_workspace_init(void *ws, int64_t t, void *stream);
+
+/* Copies the workspace bookkeeping to *out.  Synchronizes `stream` (waits for queued steps). */
+int zero_read_result(const void *ws, zero_step_result_t *out, void *stream);
+
+/* ------------------------------------------------------------------ building blocks */
+
+/* Starts a step: clears the pending overflow flag and sum of squares.  Async. */
+int zero_begin_step(void *ws, void *stream);
+
+/* Reduce-scatter of gradients ([P1] §二 ZeRO-2: gradients are reduced and scattered to the
+ * owning ranks; [P3] backward: ReduceScatter).  For every global index i in [lo, hi):
+ *     g[i] = (grads[0][i] + grads[1][i] + ... + grads[Nd-1][i]) * inv      (fp32, rank order)
+ * with inv = 1/(Nd*loss_scale) (grad_average) or 1/loss_scale, written to grad_out[i] (fp32;
+ * element i belongs to rank i/S's shard).  grads: host array of Nd device pointers to replicas
+ * of `dtype` (ZERO_BF16 / ZERO_FP16) that cover [lo, hi).  Adds whether any g is inf/NaN and
+ * sum(g^2) to the pending values in the workspace.  Only hp->loss_scale and hp->grad_average
+ * are read.  0 <= lo <= hi; 1 <= Nd <= ZERO_MAX_ND.  Async. */
+int zero_reduce_scatter(const uint16_t *const *grads, int dtype, int Nd, int64_t lo, int64_t hi,
+                        const zero_hparams_t *hp, float *grad_out, void *ws, void *stream);
+
+/* Adam/AdamW on a shard ([P1] §二: each rank runs the optimizer step on the parameters it
+ * holds; [P2] "ZeRO Stage 1"; [P3] parameter update).  Unless the pending overflow flag is set
+ * (then nothing is written), for every i in [lo, hi), in fp32 with t = completed updates + 1:
+ *     p = p * (1 - lr*wd)
+ *     m = b1*m + (1-b1)*g
+ *     v = b2*v + ((1-b2)*g)*g
+ *     p = p - (lr/(1-b1^t)) * (m / (sqrt(v)/sqrt(1-b2^t) + eps))
+ * on master/exp_avg/exp_avg_sq[i] in place, with g = grad[i].  The scalars in parentheses are
+ * evaluated in double and rounded once to fp32.  If param_out is not NULL, param_out[i] =
+ * bf16(p) (round to nearest even; the ZeRO-3 weight shard).  Does not advance t (see
+ * zero_end_step).  Async. */
+int zero_adam_shard(float *master, float *exp_avg, float *exp_avg_sq, const float *grad,
+                    int64_t lo, int64_t hi, const zero_hparams_t *hp, uint16_t *param_out,
+                    void *ws, void *stream);
+
+/* All-gather of the updated weights ([P1] §二 ZeRO-1: the updated parameters are all-gathered
+ * to every rank; [P3] forward: AllGather): replicas[r][i] = bf16(master[i]) for every rank
+ * r < Nd and i in [lo, hi).  gate = ZERO_GATE_ALWAYS or ZERO_GATE_NO_OVERFLOW (then nothing
+ * is written if the pending overflow flag is set; ws may be NULL with ZERO_GATE_ALWAYS).
+ * Async. */
+int zero_allgather(const float *master, uint16_t *const *replicas, int Nd, int64_t lo,
+                   int64_t hi, int gate, const void *ws, void *stream);
+
+/* Ends a step: if the pending overflow flag is clear, t = t + 1, otherwise the skip count
+ * grows; the pending values become the "last step" values of zero_read_result.  Async. */
+int zero_end_step(void *ws, void *stream);
+
+/* ZeRO-3 just-in-time gather of one layer ([P1] §三: before a layer runs, its full parameters
+ * are all-gathered from the ranks holding the shards and freed after use; [P2] "ZeRO Stage 3";
+ * [P3] forward).  shards: Nd device pointers, shard r holds elements [r*S, (r+1)*S) of the
+ * layer (S = ceil(L/Nd); the last shards may be partly or wholly padding).  Writes the L
+ * elements out[o][j] = shards[j/S][j%S] for every one of the nout (1..ZERO_MAX_ND) output
+ * buffers (one per rank that receives the layer).  Async. */
+int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_t *const *out,
+                       int nout, void *stream);
+
+/* ------------------------------------------------------------------ one whole step */
+
+/* One optimizer step of ZeRO stage 1, 2 or 3 ([P1] §二 and §三; [P2] "ZeRO Stage 1/2/3").
+ *   stage 1/2, ZERO_FUSED (default): reduce-scatter + unscale + overflow check + Adam + bf16
+ *     cast + all-gather in one pass over each bucket [k*bucket, (k+1)*bucket) of [0, N)
+ *     (bucket = 0: one bucket).  The pass reads state copy `live` and writes copy 1-live and
+ *     the Nd weight replicas; when the step ends without overflow the copies swap, otherwise
+ *     the replicas are rewritten from the unchanged state.  Stages 1 and 2 compute the same
+ *     values (they differ in what a real cluster keeps in memory, see zero_memory_estimate).
+ *   stage 1/2, ZERO_TWO_PASS: reduce-scatter into grad_shard, then (if no overflow) Adam in
+ *     place on copy 0 fused with the cast and the all-gather.
+ *   stage 3: N elements in layers of `bucket` elements (the last may be shorter; bucket = 0
+ *     means one layer), each padded to a multiple of Nd.  For each layer: gather its bf16
+ *     weights from param_shard into params[r] (every rank), reduce-scatter its gradient
+ *     replicas into grad_shard; after the last layer, if no overflow, Adam in place on copy 0
+ *     and param_shard = bf16(master).
+ * Every path skips the whole update (state, weights, t) when any reduced gradient element is
+ * inf or NaN.  Asynchronous: call zero_read_result to learn whether the step was skipped. */
+int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t *st,
+              const zero_hparams_t *hp, void *stream);
+
+/* Tracing hook.  Registers two cudaEvent_t handles (passed as void*) for the next zero_step
+ * call on this thread: `start_event` is recorded on its stream just before the first kernel
+ * that reads gradients and `stop_event` just after the last kernel that writes state (for
+ * ZERO_FUSED: around the fused kernels, before the overflow-repair check).  One-shot: the
+ * registration is cleared once each event is recorded.  NULL clears.  The events stay owned
+ * by the caller.  Always returns ZERO_OK. */
+int zero_profile_events(void *start_event, void *stop_event);
+
+/* ------------------------------------------------------------------ accounting (host only) */
+
+/* Per-GPU model-state memory ([P1] §二 code: bytes_per_param for the 16-bit weights and again
+ * for the gradients, bytes_per_opt_state for Adam's fp32 copy + m + v).  out[0] plain data
+ * parallelism, out[1] ZeRO-1 (optimizer state / Nd), out[2] ZeRO-2 (also gradients / Nd),
+ * out[3] ZeRO-3 (everything / Nd).  N >= 0, Nd >= 1. */
+int zero_memory_estimate(double N, int Nd, int bytes_per_param, int bytes_per_opt_state,
+                         zero_mem_t out[4]);
+
+/* Elements each rank sends per step with ring collectives ([P1] §二, §三; [P3] core
+ * operations): stage 0 (plain data parallelism) and stages 1/2 send 2(Nd-1)/Nd*N, stage 3
+ * 3(Nd-1)/Nd*N (1.5x).  Returns a negative value for a bad stage or Nd < 1. */
+double zero_comm_volume(int stage, double N, int Nd);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_H */

@@ -1,10 +1,9 @@
-"""Seeded synthetic inputs for the ZeRO step: one counter-based generator, two implementations.
+"""Seeded synthetic inputs for the ZeRO step: one counter-based generator, three implementations.
 
 This module holds no part of the optimizer's arithmetic.  It serves both the CPU oracle and
 the CUDA path: the tests and the benchmark draw every input (gradient replicas, master
-weights, moments) from it, either on the host (``values``, numpy) or directly in device
-memory (``fill_device``, the CUDA kernel in ``synth.cu``).  Both implement the same
-definition, bit for bit, and a GPU test checks that they agree.
+weights, moments) from it, either on the host or directly in device memory, all from the
+same definition, bit for bit.
 
 Definition (SplitMix64, Steele, Lea & Flood, "Fast splittable pseudorandom number
 generators", OOPSLA 2014, with the finalizer "variant 13" of Stafford's mix functions):
@@ -26,7 +25,12 @@ mean 0, variance 1 - 2^-32.  The value kinds are (every product one fp32 multipl
     HEAVY   z * sigma, except z * tail_sigma where out(sub(seed, stream ^ TAIL), k) % tail_mod == 0
     ZERO    0
 
-and the output is cast to fp32, bf16 or fp16 with round-to-nearest-even.
+and the output is stored as fp32, as fp16 (round to nearest even) or as bf16 (the upper 16
+bits of the fp32 value, i.e. rounded toward zero).
+
+Three implementations of this one definition: ``values`` (numpy, the readable reference, used
+for sampled indices), ``fill_host`` (C, synth_host.c, for large host arrays) and
+``fill_device`` (CUDA, synth.cu).  Tests check that all three agree bit for bit.
 """
 from __future__ import annotations
 
@@ -126,16 +130,14 @@ def values_f32(kind: int, seed: int, stream: int, idx, sigma: float = 1.0,
 
 
 def to_dtype_bits(x: np.ndarray, dtype: int) -> np.ndarray:
-    """Round fp32 values to bf16 / fp16 (nearest, ties to even); returns uint16 bit patterns
-    (or the float32 array itself for F32)."""
+    """Store fp32 values as the generator's output type: uint16 bit patterns for fp16 (round to
+    nearest even) and bf16 (upper half of the fp32 word), float32 for F32."""
     if dtype == F32:
         return x.astype(np.float32)
     if dtype == FP16:
         return x.astype(np.float16).view(np.uint16)
     if dtype == BF16:
-        import torch
-        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(
-            torch.bfloat16).view(torch.int16).numpy().view(np.uint16).copy()
+        return (np.ascontiguousarray(x, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
     raise ValueError("unknown dtype %r" % dtype)
 
 
@@ -144,15 +146,27 @@ def values(kind: int, dtype: int, seed: int, stream: int, idx, sigma: float = 1.
     return to_dtype_bits(values_f32(kind, seed, stream, idx, sigma, tail_sigma, tail_mod), dtype)
 
 
-def fill_host(kind, dtype, seed, stream, n, sigma=1.0, tail_sigma=0.0, tail_mod=100,
-              first=0, chunk=1 << 22) -> np.ndarray:
-    """Values for indices first .. first+n-1 (chunked to bound temporaries)."""
+def fill_host_numpy(kind, dtype, seed, stream, n, sigma=1.0, tail_sigma=0.0, tail_mod=100,
+                    first=0, chunk=1 << 22) -> np.ndarray:
+    """Values for indices first .. first+n-1 with the numpy implementation (slow)."""
     out = np.empty(n, dtype=np.float32 if dtype == F32 else np.uint16)
     for lo in range(0, n, chunk):
         hi = min(n, lo + chunk)
         out[lo:hi] = values(kind, dtype, seed, stream, np.arange(first + lo, first + hi,
                                                                   dtype=np.int64),
                             sigma, tail_sigma, tail_mod)
+    return out
+
+
+def fill_host(kind, dtype, seed, stream, n, sigma=1.0, tail_sigma=0.0, tail_mod=100,
+              first=0) -> np.ndarray:
+    """Values for indices first .. first+n-1 with the C implementation."""
+    out = np.empty(n, dtype=np.float32 if dtype == F32 else np.uint16)
+    rc = _host_lib().synth_fill_host(out.ctypes.data, dtype, kind, seed & MASK, stream & MASK,
+                                     first, n, float(np.float32(sigma)),
+                                     float(np.float32(tail_sigma)), tail_mod)
+    if rc != 0:
+        raise ValueError("synth_fill_host rejected its arguments")
     return out
 
 
@@ -181,13 +195,41 @@ NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", 
               "-Xcompiler", "-fPIC", "-shared", "-fmad=false"]
 
 
+_HOST_SRC = os.path.join(_HERE, "synth_host.c")
+_HOST_SO = os.path.join(_HERE, "libzsynth_host.so")
+
+
 def build(force: bool = False) -> str:
     if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
         tmp = _SO + ".tmp.%d" % os.getpid()
         nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
         subprocess.run([nvcc, *NVCC_FLAGS, _SRC, "-o", tmp], check=True)
         os.replace(tmp, _SO)
+    if (force or not os.path.exists(_HOST_SO)
+            or os.path.getmtime(_HOST_SO) < os.path.getmtime(_HOST_SRC)):
+        tmp = _HOST_SO + ".tmp.%d" % os.getpid()
+        subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-std=c11", "-fPIC", "-shared",
+                        _HOST_SRC, "-o", tmp], check=True)
+        os.replace(tmp, _HOST_SO)
     return _SO
+
+
+_host = None
+
+
+def _host_lib():
+    global _host
+    if _host is None:
+        if not os.path.exists(_HOST_SO):
+            build()
+        L = ctypes.CDLL(_HOST_SO)
+        L.synth_fill_host.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int64,
+                                      ctypes.c_int64, ctypes.c_float, ctypes.c_float,
+                                      ctypes.c_uint32]
+        L.synth_fill_host.restype = ctypes.c_int
+        _host = L
+    return _host
 
 
 _dev = None

@@ -3,7 +3,7 @@
 // Test and benchmark infrastructure: it writes synthetic gradient replicas, master weights
 // and moments straight into device memory so that multi-gigabyte inputs need no host
 // round trip.  It holds none of the optimizer's arithmetic.  The definition (SplitMix64
-// outputs, Irwin-Hall(12) sum of 16-bit fields, value kinds, round-to-nearest-even output)
+// outputs, Irwin-Hall(12) sum of 16-bit fields, value kinds, output types)
 // is documented in synth/__init__.py; this file implements it bit for bit.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -59,7 +59,7 @@ __global__ void fill_kernel(const FillArgs a) {
     } else if (a.dtype == 1) {
       static_cast<__half*>(a.dst)[e] = __float2half_rn(x);
     } else {
-      static_cast<__nv_bfloat16*>(a.dst)[e] = __float2bfloat16_rn(x);
+      static_cast<uint16_t*>(a.dst)[e] = (uint16_t)(__float_as_uint(x) >> 16);  // upper half
     }
   }
 }

@@ -8,6 +8,13 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_sessionstart(session):
+    # compile the CUDA library, the device input generator and the oracle before collection
+    # (nvcc and gcc cross-compile; no GPU needed)
+    import __graft_entry__
+    __graft_entry__.build_libraries()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200); run with -m gpu")
     config.addinivalue_line("markers", "slow: long-running CPU test")

@@ -1,0 +1,107 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared entry point, and
+its host-only functions (partition, accounting, argument validation) behave."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def zero():
+    import zero_sharded_optimizer_03_b200 as z  # built by conftest at session start
+    return z
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "zero.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(zero3?_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ["zero_partition", "zero_reduce_scatter", "zero_adam_shard", "zero_allgather",
+                 "zero_step", "zero3_gather_layer", "zero_memory_estimate", "zero_comm_volume"]:
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(zero):
+    out = subprocess.run(["nm", "-D", "--defined-only", zero.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(zero.LIB_PATH)
+    for n in declared_functions():
+        assert getattr(lib, n) is not None
+
+
+def test_partition_matches_oracle(zero):
+    for Nd in (1, 2, 3, 4, 7, 8, 16, 64):
+        for N in list(range(0, 70)) + [1_000_003, 124_439_808, 6_476_005_376]:
+            p = zero.zero_partition(N, Nd)
+            assert (p.S, p.Np, p.pad) == oracle.partition(N, Nd)
+            assert p.N == N and p.Nd == Nd
+
+
+def test_partition_rejects(zero):
+    for N, Nd in [(-1, 4), (10, 0), (10, 65)]:
+        with pytest.raises(zero.ZeroError) as e:
+            zero.zero_partition(N, Nd)
+        assert e.value.code == -1
+    assert "Nd=65" in zero.lib.zero_last_error().decode()
+
+
+def test_accounting_matches_oracle(zero):
+    for N, Nd, bpp, bpo in [(175e9, 64, 2, 12), (7e9, 8, 2, 4), (1e9, 1, 4, 8), (0.0, 3, 2, 12)]:
+        a = zero.zero_memory_estimate(N, Nd, bpp, bpo)
+        b = oracle.memory_estimate(N, Nd, bpp, bpo)
+        for stage in b:
+            for k in b[stage]:
+                assert a[stage][k] == pytest.approx(b[stage][k], rel=1e-14, abs=0)
+    for stage in range(4):
+        for Nd in (1, 2, 8, 64):
+            assert zero.zero_comm_volume(stage, 1e9, Nd) == pytest.approx(
+                oracle.comm_volume(stage, 1e9, Nd), rel=1e-15)
+    assert zero.zero_comm_volume(4, 1.0, 2) < 0 and zero.zero_comm_volume(1, 1.0, 0) < 0
+
+
+def test_workspace_and_version(zero):
+    assert 256 < zero.zero_workspace_bytes() < (1 << 20)
+    assert "sm_100a" in zero.zero_version()
+
+
+def test_entry_points_validate_before_touching_the_device(zero):
+    hp = zero.hparams(1e-3)
+    st = zero.zero_state_t()
+    cases = [
+        lambda: zero.zero_step(4, 4, 10, 0, st, hp),                      # bad stage
+        lambda: zero.zero_step(1, 0, 10, 0, st, hp),                      # bad Nd
+        lambda: zero.zero_step(1, 4, -1, 0, st, hp),                      # bad N
+        lambda: zero.zero_step(1, 4, 10, 0, st, zero.hparams(1e-3, beta1=1.0)),
+        lambda: zero.zero_step(1, 4, 10, 0, st, zero.hparams(1e-3, eps=0.0)),
+        lambda: zero.zero_step(1, 4, 10, 0, st, zero.hparams(1e-3, loss_scale=0.0)),
+        lambda: zero.zero_step(1, 4, 10, 0, st, hp),                      # NULL workspace
+        lambda: zero.zero_reduce_scatter([0] * 4, 0, 4, 0, 8, hp, 0, 0),  # NULL pointers
+        lambda: zero.zero_reduce_scatter([8] * 4, 2, 4, 0, 8, hp, 16, 16),  # bad dtype
+        lambda: zero.zero_reduce_scatter([16] * 4, 0, 4, 5, 4, hp, 16, 16),  # hi < lo
+        lambda: zero.zero_adam_shard(0, 0, 0, 0, 0, 8, hp, None, 0),
+        lambda: zero.zero_allgather(16, [16] * 2, 2, 0, 8, 7, 16),          # bad gate
+        lambda: zero.zero_allgather(16, [16] * 2, 2, 0, 8, 1, None),        # gate needs ws
+        lambda: zero.zero3_gather_layer([16] * 2, 2, 8, [16] * 2 * 33),     # nout too large
+        lambda: zero.zero3_gather_layer([16] * 2, 2, -1, [16]),
+        lambda: zero.zero_workspace_init(None, 0),
+        lambda: zero.zero_workspace_init(16, -3),
+    ]
+    for k, call in enumerate(cases):
+        with pytest.raises(zero.ZeroError) as e:
+            call()
+        assert e.value.code == zero.ZERO_EINVAL, k
+        assert zero.lib.zero_last_error().decode() != ""

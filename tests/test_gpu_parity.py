@@ -1,0 +1,570 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Tolerances (fixed by the method's precision: fp32 state, bf16 weights): fp32 master / m / v
+within max relative error 1e-6 (expected 0: both sides use the same fp32 operation order and
+rank-order summation), bf16 weights within 1 ulp (expected 0), overflow flag, step counter
+and shard / padding layout exact, sum of squares within 1e-5 relative (summation order
+differs).  Small and ragged sizes are compared in full; the five workloads at full size are
+compared on sampled elements the oracle evaluates one by one (plus properties that hold at
+any size).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import zero_sharded_optimizer_03_b200 as zero
+from _gpu import (HP_C1, HP_C2, HP_C3, HP_C4, HP_C5, LLAMA7B_LAYER, SEED, SampledOracle, at,
+                  assert_bf16_close, assert_f32_close, boundaries, f32, fill, free, grads_at,
+                  put_bits, sample_indices, stream, u16)
+
+pytestmark = pytest.mark.gpu
+
+DT = {zero.ZERO_BF16: (oracle.BF16, synth.BF16), zero.ZERO_FP16: (oracle.FP16, synth.FP16)}
+
+
+def _init_state(buf, N, t0=0, m_kind=synth.ZERO, v_kind=synth.ZERO, m_sigma=0.0, v_sigma=0.0):
+    fill(buf.master[0], synth.NORMAL, synth.F32, synth.MASTER_STREAM, n=N, sigma=0.02)
+    if m_kind != synth.ZERO:
+        fill(buf.exp_avg[0], m_kind, synth.F32, synth.M_STREAM, n=N, sigma=m_sigma)
+        fill(buf.exp_avg_sq[0], v_kind, synth.F32, synth.V_STREAM, n=N, sigma=v_sigma)
+    buf.init_workspace(t0)
+    buf.sync_params_from_master()
+
+
+def _host_state(N, Np, m_kind=synth.ZERO, v_kind=synth.ZERO, m_sigma=0.0, v_sigma=0.0):
+    p = np.zeros(Np, np.float32)
+    m = np.zeros(Np, np.float32)
+    v = np.zeros(Np, np.float32)
+    p[:N] = synth.fill_host(synth.NORMAL, synth.F32, SEED, synth.MASTER_STREAM, N, sigma=0.02)
+    if m_kind != synth.ZERO:
+        m[:N] = synth.fill_host(m_kind, synth.F32, SEED, synth.M_STREAM, N, sigma=m_sigma)
+        v[:N] = synth.fill_host(v_kind, synth.F32, SEED, synth.V_STREAM, N, sigma=v_sigma)
+    return p, m, v
+
+
+def _compare_full(buf, om, mm, vm, oreps, t, ss, tag):
+    res = buf.result()
+    assert res["step"] == t, (tag, res)
+    live = buf.live()
+    assert_f32_close(f32(buf.master[live]), om, tag + " master")
+    assert_f32_close(f32(buf.exp_avg[live]), mm, tag + " exp_avg")
+    assert_f32_close(f32(buf.exp_avg_sq[live]), vm, tag + " exp_avg_sq")
+    for r, rep in enumerate(oreps):
+        assert_bf16_close(u16(buf.params[r]), rep, "%s replica %d" % (tag, r))
+    if ss is not None and ss > 0:
+        assert abs(res["grad_sumsq"] - ss) <= 1e-5 * ss, (res["grad_sumsq"], ss)
+    return res
+
+
+# ----------------------------------------------------------------------------- generator
+
+@pytest.mark.parametrize("kind,dtype", [(synth.NORMAL, synth.BF16), (synth.NORMAL, synth.FP16),
+                                        (synth.NORMAL, synth.F32), (synth.ABS, synth.F32),
+                                        (synth.SQUARE, synth.F32), (synth.HEAVY, synth.BF16)])
+def test_device_generator_matches_host(kind, dtype):
+    n, first = 300_001, 12_345
+    tdt = {synth.BF16: torch.bfloat16, synth.FP16: torch.float16, synth.F32: torch.float32}[dtype]
+    t = torch.empty(n, dtype=tdt, device="cuda")
+    fill(t, kind, dtype, 77, sigma=1e-3, tail_sigma=1.0, first=first)
+    want = synth.fill_host(kind, dtype, SEED, 77, n, sigma=1e-3, tail_sigma=1.0, first=first)
+    got = u16(t) if dtype != synth.F32 else t.cpu().numpy()
+    assert got.tobytes() == want.tobytes()
+
+
+# ----------------------------------------------------------------------------- config 1, full
+
+@pytest.mark.parametrize("flags", [zero.ZERO_FUSED, zero.ZERO_TWO_PASS])
+@pytest.mark.parametrize("stage", [1, 2])
+def test_config1_zero2_single_step_full(stage, flags):
+    """N = 1,000,003 (padded to ceil(N/4)), Nd = 4, bf16 grads ~N(0,1e-3) per rank, master
+    ~N(0,0.02), m = v = 0, Adam lr 1e-3 (wd 0), step 1: every element compared."""
+    Nd, N = 4, 1_000_003
+    buf = zero.ZeroBuffers(stage, Nd, N, flags=flags)
+    _init_state(buf, N)
+    S, Np, pad = oracle.partition(N, Nd)
+    assert (buf.Np, pad) == (Np, 1)
+    om, mm, vm = _host_state(N, Np)
+    grads = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(1, r), N,
+                             sigma=1e-3) for r in range(Nd)]
+    for r in range(Nd):
+        fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(1, r), sigma=1e-3)
+    buf.step(zero.hparams(**HP_C1))
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t, ovf, ss = oracle.zero12_step(Nd, N, 0, oracle.BF16, grads, om, mm, vm, oreps, HP_C1, 0)
+    res = _compare_full(buf, om, mm, vm, oreps, t, ss, "c1")
+    assert res["overflow"] == 0 and res["skipped"] == 0
+    live = buf.live()
+    # every rank's shard view holds exactly that rank's elements; the padding stays zero
+    mast = f32(buf.master[live])
+    for r in range(Nd):
+        lo, hi = r * S, min((r + 1) * S, N)
+        assert mast[lo:hi].tobytes() == om[lo:hi].tobytes()
+    assert (mast[N:] == 0).all() and (f32(buf.exp_avg[live])[N:] == 0).all()
+    # step 1 of Adam moves every weight by at most lr
+    assert np.abs(mast[:N] - _host_state(N, Np)[0][:N]).max() <= 1e-3 * (1 + 1e-6)
+    del buf
+    free()
+
+
+# ----------------------------------------------------------------------------- small / ragged
+
+CASES = [(0, 4), (1, 1), (1, 4), (7, 3), (8, 8), (9, 2), (15, 64), (17, 5), (1000, 3),
+         (4097, 8), (65_537, 7), (262_147, 16)]
+
+
+@pytest.mark.parametrize("N,Nd", CASES)
+@pytest.mark.parametrize("gdt", [zero.ZERO_BF16, zero.ZERO_FP16])
+@pytest.mark.parametrize("flags,bucket", [(zero.ZERO_FUSED, 0), (zero.ZERO_FUSED, 1001),
+                                          (zero.ZERO_TWO_PASS, 0), (zero.ZERO_TWO_PASS, 777)])
+def test_small_ragged_three_steps(N, Nd, gdt, flags, bucket):
+    odt, sdt = DT[gdt]
+    hp = dict(HP_C3) if gdt == zero.ZERO_FP16 else dict(HP_C2)
+    sigma = 1e-4 * 1024 if gdt == zero.ZERO_FP16 else 1e-3
+    buf = zero.ZeroBuffers(2, Nd, N, grad_dtype=gdt, flags=flags)
+    _init_state(buf, N)
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t = 0
+    ss = None
+    for k in range(1, 4):
+        grads = [synth.fill_host(synth.NORMAL, sdt, SEED, synth.grad_stream(k, r), N,
+                                 sigma=sigma) for r in range(Nd)]
+        for r in range(Nd):
+            if N:
+                fill(buf.grads[r], synth.NORMAL, sdt, synth.grad_stream(k, r), n=N, sigma=sigma)
+        buf.step(zero.hparams(**hp), bucket=bucket)
+        t, ovf, ss = oracle.zero12_step(Nd, N, bucket, odt, grads, om, mm, vm, oreps, hp, t)
+    _compare_full(buf, om, mm, vm, oreps, t, ss, "N=%d Nd=%d" % (N, Nd))
+    del buf
+    free()
+
+
+def test_unaligned_views_take_the_scalar_path():
+    """Buffers that start 2 or 4 bytes past a 16-byte boundary are legal and give the same
+    results as aligned ones."""
+    Nd, N = 3, 5003
+    hp = dict(HP_C2)
+    S, Np, _ = oracle.partition(N, Nd)
+    big = [torch.zeros(N + 1, dtype=torch.bfloat16, device="cuda") for _ in range(2 * Nd)]
+    st_big = [torch.zeros(Np + 1, dtype=torch.float32, device="cuda") for _ in range(6)]
+    grads = [b[1:] for b in big[:Nd]]
+    reps = [b[1:] for b in big[Nd:]]
+    states = [b[1:] for b in st_big]
+    ws = torch.zeros(zero.zero_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    st = zero.zero_state_t()
+    st.grad_dtype = zero.ZERO_BF16
+    st.flags = zero.ZERO_FUSED
+    for r in range(Nd):
+        st.grads[r] = grads[r].data_ptr()
+        st.params[r] = reps[r].data_ptr()
+    for k in range(2):
+        st.master[k] = states[k].data_ptr()
+        st.exp_avg[k] = states[2 + k].data_ptr()
+        st.exp_avg_sq[k] = states[4 + k].data_ptr()
+    st.workspace = ws.data_ptr()
+    om, mm, vm = _host_state(N, Np)
+    states[0].copy_(torch.from_numpy(om))
+    zero.zero_workspace_init(ws.data_ptr(), 0, stream())
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t = 0
+    for k in range(1, 3):
+        hg = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(k, r), N,
+                              sigma=1e-3) for r in range(Nd)]
+        for r in range(Nd):
+            grads[r].view(torch.int16).copy_(torch.from_numpy(hg[r].view(np.int16)))
+        zero.zero_step(1, Nd, N, 0, st, zero.hparams(**hp), stream())
+        t, _, _ = oracle.zero12_step(Nd, N, 0, oracle.BF16, hg, om, mm, vm, oreps, hp, t)
+    live = zero.zero_read_result(ws.data_ptr(), stream())["live"]
+    assert_f32_close(states[live].cpu().numpy(), om, "unaligned master")
+    assert_f32_close(states[4 + live].cpu().numpy(), vm, "unaligned exp_avg_sq")
+    for r in range(Nd):
+        assert_bf16_close(u16(reps[r]), oreps[r], "unaligned replica")
+
+
+def test_stage1_and_stage2_identical():
+    Nd, N = 8, 300_001
+    outs = []
+    for stage in (1, 2):
+        buf = zero.ZeroBuffers(stage, Nd, N)
+        _init_state(buf, N)
+        for k in (1, 2):
+            for r in range(Nd):
+                fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(k, r), sigma=1e-3)
+            buf.step(zero.hparams(**HP_C2))
+        live = buf.live()
+        outs.append((f32(buf.master[live]).tobytes(), u16(buf.params[5]).tobytes()))
+        del buf
+    assert outs[0] == outs[1]
+    free()
+
+
+def test_bucketed_equals_unbucketed_and_repeatable():
+    Nd, N = 4, 1_000_003
+    outs = []
+    for bucket in (0, 100_000, 77_777, 1_000_003, 3):
+        buf = zero.ZeroBuffers(2, Nd, N)
+        _init_state(buf, N)
+        for r in range(Nd):
+            fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(1, r), sigma=1e-3)
+        buf.step(zero.hparams(**HP_C2), bucket=bucket)
+        live = buf.live()
+        outs.append((f32(buf.master[live]).tobytes(), f32(buf.exp_avg_sq[live]).tobytes(),
+                     u16(buf.params[3]).tobytes()))
+        del buf
+    assert all(o == outs[0] for o in outs)
+    free()
+
+
+# ----------------------------------------------------------------------------- overflow skip
+
+@pytest.mark.parametrize("flags", [zero.ZERO_FUSED, zero.ZERO_TWO_PASS])
+@pytest.mark.parametrize("bad", [0x7F80, 0xFF80, 0x7FC1, "pair"])
+def test_overflow_skips_then_recovers(flags, bad):
+    Nd, N = 4, 200_003
+    hp = dict(HP_C2)
+    buf = zero.ZeroBuffers(2, Nd, N, flags=flags)
+    _init_state(buf, N, t0=10)
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    oreps = [oracle.f32_to_bf16(om[:N]) for _ in range(Nd)]
+    t = 10
+    # step A: clean
+    hg = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(1, r), N, sigma=1e-3)
+          for r in range(Nd)]
+    for r in range(Nd):
+        fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(1, r), sigma=1e-3)
+    buf.step(zero.hparams(**hp))
+    t, _, _ = oracle.zero12_step(Nd, N, 0, oracle.BF16, hg, om, mm, vm, oreps, hp, t)
+    live = buf.live()
+    snap = [f32(buf.master[live]).tobytes(), f32(buf.exp_avg[live]).tobytes(),
+            f32(buf.exp_avg_sq[live]).tobytes()] + [u16(p).tobytes() for p in buf.params]
+    # step B: one non-finite gradient element somewhere -> the whole step is skipped
+    hg = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(2, r), N, sigma=1e-3)
+          for r in range(Nd)]
+    for r in range(Nd):
+        fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(2, r), sigma=1e-3)
+    if bad == "pair":  # +inf and -inf at the same element of two ranks: the sum is NaN
+        for r, bits in ((1, 0x7F80), (2, 0xFF80)):
+            put_bits(buf.grads[r], 12_345, bits)
+            hg[r][12_345] = bits
+    else:
+        put_bits(buf.grads[3], N - 1, bad)
+        hg[3][N - 1] = bad
+    buf.step(zero.hparams(**hp))
+    t2, ovf, _ = oracle.zero12_step(Nd, N, 0, oracle.BF16, hg, om, mm, vm, oreps, hp, t)
+    assert ovf == 1 and t2 == t
+    res = buf.result()
+    assert res["overflow"] == 1 and res["skipped"] == 1 and res["step"] == t
+    live = buf.live()
+    now = [f32(buf.master[live]).tobytes(), f32(buf.exp_avg[live]).tobytes(),
+           f32(buf.exp_avg_sq[live]).tobytes()] + [u16(p).tobytes() for p in buf.params]
+    assert now == snap, "a skipped step changed the state or the replicas"
+    # step C: clean again, continues from the unchanged state with t + 1
+    hg = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(3, r), N, sigma=1e-3)
+          for r in range(Nd)]
+    for r in range(Nd):
+        fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(3, r), sigma=1e-3)
+    buf.step(zero.hparams(**hp))
+    t, _, ss = oracle.zero12_step(Nd, N, 0, oracle.BF16, hg, om, mm, vm, oreps, hp, t)
+    res = _compare_full(buf, om, mm, vm, oreps, t, ss, "after skip")
+    assert res["overflow"] == 0 and res["skipped"] == 1 and res["step"] == 12
+    del buf
+    free()
+
+
+# ----------------------------------------------------------------------------- building blocks
+
+def test_building_blocks_two_pass_matches_oracle():
+    """begin -> reduce_scatter (per rank's shard) -> adam (per shard) -> allgather -> end."""
+    Nd, N = 5, 123_457
+    hp = dict(HP_C3)
+    S, Np, _ = oracle.partition(N, Nd)
+    sigma = 0.1024
+    grads = [torch.zeros(N, dtype=torch.float16, device="cuda") for _ in range(Nd)]
+    reps = [torch.zeros(N, dtype=torch.bfloat16, device="cuda") for _ in range(Nd)]
+    p = torch.zeros(Np, device="cuda")
+    m = torch.zeros(Np, device="cuda")
+    v = torch.zeros(Np, device="cuda")
+    gsh = torch.zeros(Np, device="cuda")
+    ws = torch.zeros(zero.zero_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    om, mm, vm = _host_state(N, Np)
+    p.copy_(torch.from_numpy(om))
+    zero.zero_workspace_init(ws.data_ptr(), 0, stream())
+    chp = zero.hparams(**hp)
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t = 0
+    for k in (1, 2):
+        hg = [synth.fill_host(synth.NORMAL, synth.FP16, SEED, synth.grad_stream(k, r), N,
+                              sigma=sigma) for r in range(Nd)]
+        for r in range(Nd):
+            fill(grads[r], synth.NORMAL, synth.FP16, synth.grad_stream(k, r), sigma=sigma)
+        zero.zero_begin_step(ws.data_ptr(), stream())
+        gp = [g.data_ptr() for g in grads]
+        for r in range(Nd):  # every rank reduce-scatters its own shard
+            lo, hi = min(r * S, N), min((r + 1) * S, N)
+            zero.zero_reduce_scatter(gp, zero.ZERO_FP16, Nd, lo, hi, chp, gsh.data_ptr(),
+                                     ws.data_ptr(), stream())
+        for r in range(Nd):
+            lo, hi = min(r * S, N), min((r + 1) * S, N)
+            zero.zero_adam_shard(p.data_ptr(), m.data_ptr(), v.data_ptr(), gsh.data_ptr(), lo, hi,
+                                 chp, None, ws.data_ptr(), stream())
+        zero.zero_allgather(p.data_ptr(), [x.data_ptr() for x in reps], Nd, 0, N,
+                            zero.ZERO_GATE_NO_OVERFLOW, ws.data_ptr(), stream())
+        res_mid = zero.zero_read_result(ws.data_ptr(), stream())
+        zero.zero_end_step(ws.data_ptr(), stream())
+        t, ovf, ss = oracle.zero12_step(Nd, N, 0, oracle.FP16, hg, om, mm, vm, oreps, hp, t)
+        g_or, _, _ = oracle.reduce_scatter(Nd, N, oracle.FP16, hg, hp)
+        assert_f32_close(gsh.cpu().numpy(), g_or, "reduced gradient shard")
+        assert abs(res_mid["pending_sumsq"] - ss) <= 1e-5 * ss
+    res = zero.zero_read_result(ws.data_ptr(), stream())
+    assert res["step"] == 2 and res["overflow"] == 0
+    assert_f32_close(p.cpu().numpy(), om, "master")
+    assert_f32_close(m.cpu().numpy(), mm, "exp_avg")
+    assert_f32_close(v.cpu().numpy(), vm, "exp_avg_sq")
+    for r in range(Nd):
+        assert_bf16_close(u16(reps[r]), oreps[r], "replica")
+
+
+def test_empty_step_advances_t():
+    buf = zero.ZeroBuffers(2, 4, 0)
+    buf.init_workspace(5)
+    buf.step(zero.hparams(**HP_C1))
+    res = buf.result()
+    assert res["step"] == 6 and res["overflow"] == 0 and res["grad_sumsq"] == 0.0
+
+
+# ----------------------------------------------------------------------------- ZeRO-3
+
+@pytest.mark.parametrize("L,Nd,nout", [(202_375, 8, 8), (1001, 3, 1), (7, 4, 2), (64, 64, 3),
+                                       (25_296_896 // 64, 8, 8)])
+def test_gather_layer_full(L, Nd, nout):
+    S, Np, _ = oracle.partition(L, Nd)
+    flat = torch.zeros(Np, dtype=torch.bfloat16, device="cuda")
+    fill(flat, synth.NORMAL, synth.BF16, 99, n=L, sigma=0.02)
+    shards = [flat[r * S:(r + 1) * S] for r in range(Nd)]
+    outs = [torch.zeros(L, dtype=torch.bfloat16, device="cuda") for _ in range(nout)]
+    zero.zero3_gather_layer([s.data_ptr() for s in shards], Nd, L, [o.data_ptr() for o in outs],
+                            stream())
+    want = oracle.zero3_gather(Nd, L, [u16(s) for s in shards])
+    for o in outs:
+        assert u16(o).tobytes() == want.tobytes()
+
+
+@pytest.mark.parametrize("layer_len,N,Nd", [(1000, 5333, 3), (4096, 4096 * 3, 8),
+                                            (12_345, 12_345 * 2 + 17, 4)])
+def test_zero3_step_matches_oracle(layer_len, N, Nd):
+    """zero_step(stage=3): per-layer gather from the bf16 shards, per-layer reduce-scatter,
+    then Adam on every shard and the bf16 shard update; three steps, every element."""
+    buf = zero.ZeroBuffers(3, Nd, N, layer_len=layer_len, per_layer_buffers=True)
+    sizes = buf.layer_sizes
+    hp = dict(HP_C4)
+    total = buf.Np
+    om = np.zeros(total, np.float32)
+    off = 0
+    for l, (Ll, Lp) in enumerate(zip(sizes, buf.layer_padded)):
+        om[off:off + Ll] = synth.fill_host(synth.NORMAL, synth.F32, SEED, 1000 + l, Ll, sigma=0.02)
+        off += Lp
+    buf.master[0].copy_(torch.from_numpy(om))
+    buf.init_workspace(0)
+    buf.sync_params_from_master()
+    mm = np.zeros(total, np.float32)
+    vm = np.zeros(total, np.float32)
+    sh16 = oracle.f32_to_bf16(om)
+    assert u16(buf.param_shard).tobytes() == sh16.tobytes()
+    t = 0
+    for k in (1, 2, 3):
+        hgrads, gathered = [], []
+        for l, Ll in enumerate(sizes):
+            for r in range(Nd):
+                hg = synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(k, r, l),
+                                     Ll, sigma=1e-3)
+                hgrads.append(hg)
+                buf.grads[r][l * layer_len:l * layer_len + Ll].view(torch.int16).copy_(
+                    torch.from_numpy(hg.view(np.int16)))
+                gathered.append(np.zeros(Ll, np.uint16))
+        buf.step(zero.hparams(**hp))
+        t, ovf, ss = oracle.zero3_step(Nd, sizes, oracle.BF16, hgrads, om, mm, vm, sh16, gathered,
+                                       hp, t)
+        for l, Ll in enumerate(sizes):
+            for r in range(Nd):
+                got = u16(buf.params[r][l * layer_len:l * layer_len + Ll])
+                assert got.tobytes() == gathered[l * Nd + r].tobytes(), "gather layer %d" % l
+    res = buf.result()
+    assert res["step"] == t == 3
+    assert abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
+    assert_f32_close(f32(buf.master[0]), om, "zero3 master")
+    assert_f32_close(f32(buf.exp_avg[0]), mm, "zero3 exp_avg")
+    assert_f32_close(f32(buf.exp_avg_sq[0]), vm, "zero3 exp_avg_sq")
+    assert_bf16_close(u16(buf.param_shard), sh16, "zero3 bf16 shard")
+    del buf
+    free()
+
+
+# ----------------------------------------------------------------------------- full-size workloads
+
+def _sampled_run(stage, Nd, N, steps, hp, gdt, sigma, bucket=0, flags=zero.ZERO_FUSED,
+                 kind=synth.NORMAL, tail_sigma=0.0, t0=0, m_kind=synth.ZERO, v_kind=synth.ZERO,
+                 m_sigma=0.0, v_sigma=0.0, inject=None, n_random=100_000, extra=()):
+    odt, sdt = DT[gdt]
+    buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt, flags=flags)
+    _init_state(buf, N, t0, m_kind, v_kind, m_sigma, v_sigma)
+    inj_rank, inj_idx = inject[1] if inject else (None, None)
+    idx = sample_indices(N, n_random, list(extra) + ([inj_idx] if inject else []))
+    p0 = synth.values(synth.NORMAL, synth.F32, SEED, synth.MASTER_STREAM, idx, 0.02)
+    m0 = synth.values(m_kind, synth.F32, SEED, synth.M_STREAM, idx, m_sigma)
+    v0 = synth.values(v_kind, synth.F32, SEED, synth.V_STREAM, idx, v_sigma)
+    so = SampledOracle(idx, Nd, odt, p0, m0, v0, t0)
+    chp = zero.hparams(**hp)
+    for k in range(1, steps + 1):
+        for r in range(Nd):
+            fill(buf.grads[r], kind, sdt, synth.grad_stream(k, r), sigma=sigma,
+                 tail_sigma=tail_sigma)
+        g_en = grads_at(idx, Nd, sdt, k, sigma, kind, tail_sigma)
+        skip = bool(inject) and k == inject[0]
+        if skip:
+            put_bits(buf.grads[inj_rank], inj_idx, 0x7F80 if sdt == synth.BF16 else 0x7C00)
+            g_en[np.searchsorted(idx, inj_idx), inj_rank] = 0x7F80 if sdt == synth.BF16 else 0x7C00
+        live_before = buf.live()
+        before = at(buf.master[live_before], idx) if skip else None
+        buf.step(chp, bucket=bucket)
+        so.step(g_en, hp, skip)
+        res = buf.result()
+        assert res["overflow"] == int(skip), (k, res)
+        live = buf.live()
+        if skip:
+            assert live == live_before
+            assert at(buf.master[live], idx).tobytes() == before.tobytes()
+        assert_f32_close(at(buf.master[live], idx), so.p, "step %d master" % k)
+        assert_f32_close(at(buf.exp_avg[live], idx), so.m, "step %d exp_avg" % k)
+        assert_f32_close(at(buf.exp_avg_sq[live], idx), so.v, "step %d exp_avg_sq" % k)
+        for r in sorted({0, Nd // 2, Nd - 1}):
+            assert_bf16_close(at(buf.params[r], idx), so.out16, "step %d replica %d" % (k, r))
+    res = buf.result()
+    assert res["step"] == so.t
+    # every rank received the same weights (the all-gather is complete), whole vector
+    for r in range(1, Nd):
+        assert torch.equal(buf.params[r].view(torch.int16), buf.params[0].view(torch.int16))
+    return buf, res, so
+
+
+def test_config2_zero1_gpt2_small_ten_steps():
+    """N = 124,439,808 (GPT-2 small), Nd = 8, ZeRO-1, 10 AdamW steps (lr 6e-4, wd 0.01), fresh
+    bf16 grads ~N(0,1e-3) every step, bf16 weights all-gathered to 8 replicas each step."""
+    N, Nd = 124_439_808, 8
+    S = oracle.partition(N, Nd)[0]
+    buf, res, so = _sampled_run(1, Nd, N, 10, HP_C2, zero.ZERO_BF16, 1e-3,
+                                extra=boundaries(S, N))
+    # property at full size: the reduced gradient is the mean of 8 N(0, 1e-3) replicas, so
+    # E[sum g^2] = N * 1e-6 / 8 (the generator's variance is 1 - 2^-32)
+    assert abs(res["grad_sumsq"] / (N * 1e-6 / 8) - 1) < 0.01
+    assert res["skipped"] == 0
+    del buf
+    free()
+
+
+def test_config3_zero2_bucketed_fp16_with_overflow():
+    """N = 1.3e9 in 25M-element buckets, Nd = 16, fp16 grads ~N(0,1e-4)*1024 carrying loss
+    scale 1024 (unscaled in the kernel); +inf planted at a seeded (rank, index) on step 3,
+    which must skip that step; 5 AdamW steps."""
+    N, Nd, B = 1_300_000_000, 16, 25_000_000
+    S = oracle.partition(N, Nd)[0]
+    site = synth.inject_site(SEED, Nd, N)
+    buf, res, so = _sampled_run(2, Nd, N, 5, HP_C3, zero.ZERO_FP16, 1e-4 * 1024, bucket=B,
+                                inject=(3, site), n_random=50_000,
+                                extra=boundaries(S, N) + boundaries(B, N))
+    assert res["step"] == 4 and res["skipped"] == 1
+    del buf
+    free()
+
+
+def test_config5_wide_fan_in():
+    """N = 2^28, Nd = 64, bf16 grads ~N(0,1e-3) with 1% of values x1e3 (hash-selected), AdamW
+    step 1000 with m ~ |N(0,1e-3)|, v = N(0,1e-6)^2."""
+    N, Nd = 1 << 28, 64
+    tail = float(np.float32(1e-3 * 1e3))
+    buf, res, so = _sampled_run(2, Nd, N, 1, HP_C5, zero.ZERO_BF16, 1e-3, kind=synth.HEAVY,
+                                tail_sigma=tail, t0=999, m_kind=synth.ABS, v_kind=synth.SQUARE,
+                                m_sigma=1e-3, v_sigma=1e-6, n_random=50_000,
+                                extra=boundaries(N // Nd, N))
+    assert res["step"] == 1000 and res["overflow"] == 0
+    # E[g^2] for the mean of 64 replicas: (0.99 * 1e-6 + 0.01 * 1.0) / 64 per element
+    expect = N * (0.99e-6 + 0.01) / 64
+    assert abs(res["grad_sumsq"] / expect - 1) < 0.02
+    del buf
+    free()
+
+
+def test_target_2p28_nd8_fused():
+    N, Nd = 1 << 28, 8
+    buf, res, so = _sampled_run(2, Nd, N, 2, HP_C5, zero.ZERO_BF16, 1e-3, n_random=50_000,
+                                extra=boundaries(N // Nd, N))
+    del buf
+    free()
+
+
+def test_config4_zero3_llama7b_shaped():
+    """32 layers of q,k,v,o (4096x4096) + gate,up,down (4096x11008), bf16, Nd = 8; per layer:
+    gather the full layer from 8 shards, reduce-scatter 8 bf16 grad replicas ~N(0,1e-3) into
+    the fp32 gradient shard; then AdamW on the fp32 shards; 1 step.  Driven through the
+    building blocks with fresh gradients per layer (seeded by layer), one layer buffer reused."""
+    Nd, L, nl = 8, LLAMA7B_LAYER, 32
+    N = L * nl
+    S = oracle.partition(L, Nd)[0]
+    hp = dict(HP_C4)
+    chp = zero.hparams(**hp)
+    dev = "cuda"
+    master = torch.zeros(N, device=dev)
+    m = torch.zeros(N, device=dev)
+    v = torch.zeros(N, device=dev)
+    gsh = torch.zeros(N, device=dev)
+    sh16 = torch.zeros(N, dtype=torch.bfloat16, device=dev)
+    grads = [torch.zeros(L, dtype=torch.bfloat16, device=dev) for _ in range(Nd)]
+    gathered = [torch.zeros(L, dtype=torch.bfloat16, device=dev) for _ in range(Nd)]
+    ws = torch.zeros(zero.zero_workspace_bytes(), dtype=torch.uint8, device=dev)
+    s = stream()
+    fill(master, synth.NORMAL, synth.F32, synth.MASTER_STREAM, sigma=0.02)
+    zero.zero_allgather(master.data_ptr(), [sh16.data_ptr()], 1, 0, N, zero.ZERO_GATE_ALWAYS,
+                        None, s)
+    zero.zero_workspace_init(ws.data_ptr(), 0, s)
+    rng = np.random.default_rng(11)
+    loc = np.unique(np.concatenate([rng.integers(0, L, 4000),
+                                    np.array([0, L - 1] + boundaries(S, L))]))
+    zero.zero_begin_step(ws.data_ptr(), s)
+    samples = {}
+    for l in range(nl):
+        off = l * L
+        shards = [sh16.data_ptr() + 2 * (off + r * S) for r in range(Nd)]
+        zero.zero3_gather_layer(shards, Nd, L, [g.data_ptr() for g in gathered], s)
+        want16 = oracle.f32_to_bf16(synth.values(synth.NORMAL, synth.F32, SEED,
+                                                 synth.MASTER_STREAM, off + loc, 0.02))
+        for r in (0, Nd - 1):
+            assert at(gathered[r], loc).tobytes() == want16.tobytes(), "layer %d gather" % l
+        for r in range(Nd):
+            fill(grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(1, r, l), sigma=1e-3)
+        zero.zero_reduce_scatter([g.data_ptr() for g in grads], zero.ZERO_BF16, Nd, 0, L, chp,
+                                 gsh.data_ptr() + 4 * off, ws.data_ptr(), s)
+        samples[l] = grads_at(loc, Nd, synth.BF16, 1, 1e-3, layer=l)
+    for l in range(nl):
+        off = l * L
+        zero.zero_adam_shard(master.data_ptr() + 4 * off, m.data_ptr() + 4 * off,
+                             v.data_ptr() + 4 * off, gsh.data_ptr() + 4 * off, 0, L, chp,
+                             sh16.data_ptr() + 2 * off, ws.data_ptr(), s)
+    zero.zero_end_step(ws.data_ptr(), s)
+    res = zero.zero_read_result(ws.data_ptr(), s)
+    assert res["step"] == 1 and res["overflow"] == 0
+    assert abs(res["grad_sumsq"] / (N * 1e-6 / 8) - 1) < 0.01
+    for l in (0, 1, 17, 31):
+        gidx = l * L + loc
+        p0 = synth.values(synth.NORMAL, synth.F32, SEED, synth.MASTER_STREAM, gidx, 0.02)
+        so = SampledOracle(gidx, Nd, oracle.BF16, p0, np.zeros_like(p0), np.zeros_like(p0), 0)
+        g = so.step(samples[l], hp, False)
+        assert_f32_close(at(gsh, gidx), g, "layer %d reduced grad" % l)
+        assert_f32_close(at(master, gidx), so.p, "layer %d master" % l)
+        assert_f32_close(at(m, gidx), so.m, "layer %d exp_avg" % l)
+        assert_f32_close(at(v, gidx), so.v, "layer %d exp_avg_sq" % l)
+        assert_bf16_close(at(sh16, gidx), so.out16, "layer %d bf16 shard" % l)
+    del master, m, v, gsh, sh16, grads, gathered
+    free()

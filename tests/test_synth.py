@@ -17,7 +17,7 @@ def test_counter_based_index_addressing():
     a = synth.fill_host(synth.NORMAL, synth.F32, 1, 2, 5000, sigma=0.02)
     b = synth.values(synth.NORMAL, synth.F32, 1, 2, np.array([4999, 0, 1234]), sigma=0.02)
     assert (a[[4999, 0, 1234]] == b).all()
-    c = synth.fill_host(synth.NORMAL, synth.F32, 1, 2, 3000, sigma=0.02, first=2000, chunk=777)
+    c = synth.fill_host_numpy(synth.NORMAL, synth.F32, 1, 2, 3000, sigma=0.02, first=2000, chunk=777)
     assert (c == a[2000:]).all()
     assert not (synth.fill_host(synth.NORMAL, synth.F32, 1, 3, 100) == a[:100]).all()
 
@@ -34,13 +34,23 @@ def test_kinds():
     assert (synth.values_f32(synth.ZERO, 5, 9, idx) == 0).all()
 
 
-def test_dtypes_round_to_nearest():
+def test_output_types():
     x = synth.values_f32(synth.NORMAL, 5, 9, np.arange(1000), sigma=0.1)
     f16 = synth.to_dtype_bits(x, synth.FP16).view(np.float16)
     assert (f16 == x.astype(np.float16)).all()
     b16 = synth.to_dtype_bits(x, synth.BF16)
     back = (b16.astype(np.uint32) << 16).view(np.float32)
-    assert (np.abs(back - x) <= np.abs(x) * 2.0 ** -8).all()
+    assert (np.abs(back) <= np.abs(x)).all() and (np.abs(back - x) <= np.abs(x) * 2.0 ** -7).all()
+
+
+def test_c_and_numpy_implementations_agree():
+    for kind in (synth.NORMAL, synth.ABS, synth.SQUARE, synth.HEAVY, synth.ZERO):
+        for dtype in (synth.BF16, synth.FP16, synth.F32):
+            a = synth.fill_host(kind, dtype, 3, 41, 20_000, sigma=1e-3, tail_sigma=1.0,
+                                first=999)
+            b = synth.fill_host_numpy(kind, dtype, 3, 41, 20_000, sigma=1e-3, tail_sigma=1.0,
+                                      first=999)
+            assert a.tobytes() == b.tobytes(), (kind, dtype)
 
 
 def test_inject_site_in_range():

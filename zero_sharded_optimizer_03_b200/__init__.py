@@ -1,0 +1,307 @@
+"""Python binding of libzero.so, the B200 sharded mixed-precision Adam step (ZeRO-1/2/3).
+
+Argument marshalling only: every function forwards to the C entry point of the same name in
+``include/zero.h`` (device pointers as ints, the CUDA stream as an int handle).  All device
+work runs in the library's sm_100a kernels.  If libzero.so has not been built, importing this
+package raises ImportError: there is no fallback implementation.
+
+``ZeroBuffers`` is plumbing for callers that hold their state in torch tensors: it allocates
+the caller-owned buffers the C API expects (with torch) and fills a ``zero_state_t``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "ZeroError", "zero_partition", "zero_workspace_bytes", "zero_workspace_init",
+    "zero_read_result", "zero_begin_step", "zero_reduce_scatter", "zero_adam_shard",
+    "zero_allgather", "zero_end_step", "zero3_gather_layer", "zero_step",
+    "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events", "hparams", "ZeroBuffers",
+    "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_GATE_ALWAYS",
+    "ZERO_GATE_NO_OVERFLOW", "ZERO_MAX_ND",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzero.so")
+
+ZERO_OK, ZERO_EINVAL, ZERO_ECUDA = 0, -1, -2
+ZERO_MAX_ND = 64
+ZERO_BF16, ZERO_FP16 = 0, 1
+ZERO_FUSED, ZERO_TWO_PASS = 0, 1
+ZERO_GATE_ALWAYS, ZERO_GATE_NO_OVERFLOW = 0, 1
+
+_i64, _i32, _dbl, _P = ctypes.c_int64, ctypes.c_int32, ctypes.c_double, ctypes.c_void_p
+
+
+class zero_partition_t(ctypes.Structure):
+    _fields_ = [("N", _i64), ("Nd", _i32), ("reserved", _i32), ("S", _i64), ("Np", _i64),
+                ("pad", _i64)]
+
+
+class zero_hparams_t(ctypes.Structure):
+    _fields_ = [("lr", _dbl), ("beta1", _dbl), ("beta2", _dbl), ("eps", _dbl),
+                ("weight_decay", _dbl), ("loss_scale", _dbl), ("grad_average", _i32),
+                ("reserved", _i32)]
+
+
+class zero_step_result_t(ctypes.Structure):
+    _fields_ = [("step", _i64), ("skipped", _i64), ("overflow", _i32), ("live", _i32),
+                ("grad_sumsq", _dbl), ("pending_overflow", _i32), ("reserved", _i32),
+                ("pending_sumsq", _dbl)]
+
+
+class zero_state_t(ctypes.Structure):
+    _fields_ = [("grad_dtype", _i32), ("flags", _i32),
+                ("grads", _P * ZERO_MAX_ND), ("params", _P * ZERO_MAX_ND),
+                ("master", _P * 2), ("exp_avg", _P * 2), ("exp_avg_sq", _P * 2),
+                ("grad_shard", _P), ("param_shard", _P),
+                ("grad_layer_stride", _i64), ("param_layer_stride", _i64),
+                ("workspace", _P)]
+
+
+class zero_mem_t(ctypes.Structure):
+    _fields_ = [("optimizer_states", _dbl), ("gradients", _dbl), ("parameters", _dbl),
+                ("total", _dbl)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libzero.so is not built (expected at %s); run "
+                          "`python -m zero_sharded_optimizer_03_b200.build` or "
+                          "__graft_entry__.build()" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "zero_last_error": ([], ctypes.c_char_p),
+        "zero_version": ([], ctypes.c_char_p),
+        "zero_partition": ([_i64, ctypes.c_int, ctypes.POINTER(zero_partition_t)], ctypes.c_int),
+        "zero_workspace_bytes": ([], ctypes.c_size_t),
+        "zero_workspace_init": ([_P, _i64, _P], ctypes.c_int),
+        "zero_read_result": ([_P, ctypes.POINTER(zero_step_result_t), _P], ctypes.c_int),
+        "zero_begin_step": ([_P, _P], ctypes.c_int),
+        "zero_reduce_scatter": ([_P, ctypes.c_int, ctypes.c_int, _i64, _i64,
+                                 ctypes.POINTER(zero_hparams_t), _P, _P, _P], ctypes.c_int),
+        "zero_adam_shard": ([_P, _P, _P, _P, _i64, _i64, ctypes.POINTER(zero_hparams_t), _P,
+                             _P, _P], ctypes.c_int),
+        "zero_allgather": ([_P, _P, ctypes.c_int, _i64, _i64, ctypes.c_int, _P, _P],
+                           ctypes.c_int),
+        "zero_end_step": ([_P, _P], ctypes.c_int),
+        "zero3_gather_layer": ([_P, ctypes.c_int, _i64, _P, ctypes.c_int, _P], ctypes.c_int),
+        "zero_step": ([ctypes.c_int, ctypes.c_int, _i64, _i64, ctypes.POINTER(zero_state_t),
+                       ctypes.POINTER(zero_hparams_t), _P], ctypes.c_int),
+        "zero_memory_estimate": ([_dbl, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  ctypes.POINTER(zero_mem_t)], ctypes.c_int),
+        "zero_comm_volume": ([ctypes.c_int, _dbl, ctypes.c_int], _dbl),
+        "zero_profile_events": ([_P, _P], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
+lib = _load()
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("libzero error %d: %s" % (code, msg))
+        self.code = code
+
+
+def _check(rc: int) -> None:
+    if rc != ZERO_OK:
+        raise ZeroError(rc, lib.zero_last_error().decode())
+
+
+def _ptrs(ptrs) -> ctypes.Array:
+    arr = (_P * max(1, len(ptrs)))()
+    for k, p in enumerate(ptrs):
+        arr[k] = int(p)
+    return arr
+
+
+def hparams(lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, loss_scale=1.0,
+            grad_average=True) -> zero_hparams_t:
+    return zero_hparams_t(lr, beta1, beta2, eps, weight_decay, loss_scale,
+                          1 if grad_average else 0, 0)
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def zero_version() -> str:
+    return lib.zero_version().decode()
+
+
+def zero_partition(N: int, Nd: int) -> zero_partition_t:
+    out = zero_partition_t()
+    _check(lib.zero_partition(N, Nd, ctypes.byref(out)))
+    return out
+
+
+def zero_workspace_bytes() -> int:
+    return int(lib.zero_workspace_bytes())
+
+
+def zero_workspace_init(ws: int, t: int = 0, stream: int = 0) -> None:
+    _check(lib.zero_workspace_init(ws, t, stream))
+
+
+def zero_read_result(ws: int, stream: int = 0) -> dict:
+    out = zero_step_result_t()
+    _check(lib.zero_read_result(ws, ctypes.byref(out), stream))
+    return {k: getattr(out, k) for k, _ in zero_step_result_t._fields_ if k != "reserved"}
+
+
+def zero_begin_step(ws: int, stream: int = 0) -> None:
+    _check(lib.zero_begin_step(ws, stream))
+
+
+def zero_reduce_scatter(grads, dtype: int, Nd: int, lo: int, hi: int, hp: zero_hparams_t,
+                        grad_out: int, ws: int, stream: int = 0) -> None:
+    _check(lib.zero_reduce_scatter(_ptrs(grads), dtype, Nd, lo, hi, ctypes.byref(hp), grad_out,
+                                   ws, stream))
+
+
+def zero_adam_shard(master: int, exp_avg: int, exp_avg_sq: int, grad: int, lo: int, hi: int,
+                    hp: zero_hparams_t, param_out: int | None, ws: int, stream: int = 0) -> None:
+    _check(lib.zero_adam_shard(master, exp_avg, exp_avg_sq, grad, lo, hi, ctypes.byref(hp),
+                               param_out, ws, stream))
+
+
+def zero_allgather(master: int, replicas, Nd: int, lo: int, hi: int,
+                   gate: int = ZERO_GATE_ALWAYS, ws: int | None = None, stream: int = 0) -> None:
+    _check(lib.zero_allgather(master, _ptrs(replicas), Nd, lo, hi, gate, ws, stream))
+
+
+def zero_profile_events(start_event: int | None, stop_event: int | None) -> None:
+    _check(lib.zero_profile_events(start_event, stop_event))
+
+
+def zero_end_step(ws: int, stream: int = 0) -> None:
+    _check(lib.zero_end_step(ws, stream))
+
+
+def zero3_gather_layer(shards, Nd: int, L: int, out, stream: int = 0) -> None:
+    _check(lib.zero3_gather_layer(_ptrs(shards), Nd, L, _ptrs(out), len(out), stream))
+
+
+def zero_step(stage: int, Nd: int, N: int, bucket: int, state: zero_state_t, hp: zero_hparams_t,
+              stream: int = 0) -> None:
+    _check(lib.zero_step(stage, Nd, N, bucket, ctypes.byref(state), ctypes.byref(hp), stream))
+
+
+STAGES = ("DP", "ZeRO-1", "ZeRO-2", "ZeRO-3")
+
+
+def zero_memory_estimate(N: float, Nd: int, bytes_per_param: int = 2,
+                         bytes_per_opt_state: int = 12) -> dict:
+    out = (zero_mem_t * 4)()
+    _check(lib.zero_memory_estimate(float(N), Nd, bytes_per_param, bytes_per_opt_state, out))
+    return {STAGES[s]: {k: getattr(out[s], k) for k, _ in zero_mem_t._fields_} for s in range(4)}
+
+
+def zero_comm_volume(stage: int, N: float, Nd: int) -> float:
+    return float(lib.zero_comm_volume(stage, float(N), Nd))
+
+
+# ----------------------------------------------------------------------------- torch plumbing
+
+class ZeroBuffers:
+    """Caller-owned device buffers of one simulated ZeRO job, allocated with torch.
+
+    stage 1/2: Nd gradient replicas and Nd bf16 weight replicas of N elements; two padded
+    copies of master/exp_avg/exp_avg_sq (ZERO_FUSED ping-pongs between them) or one copy plus
+    an fp32 gradient shard (ZERO_TWO_PASS).
+    stage 3: `layers` layers of `layer_len` elements (the last may be shorter), every layer
+    padded to a multiple of Nd; one layer-sized gradient buffer and one gathered-weight
+    buffer per rank (reused for every layer unless per_layer_buffers is set).
+    """
+
+    def __init__(self, stage: int, Nd: int, N: int, grad_dtype: int = ZERO_BF16,
+                 flags: int = ZERO_FUSED, layer_len: int = 0, per_layer_buffers: bool = False,
+                 device: str = "cuda"):
+        import torch
+        self.torch = torch
+        self.stage, self.Nd, self.N, self.flags = stage, Nd, N, flags
+        self.grad_dtype = grad_dtype
+        gdt = torch.bfloat16 if grad_dtype == ZERO_BF16 else torch.float16
+        f32 = dict(dtype=torch.float32, device=device)
+        self.ws = torch.zeros(zero_workspace_bytes(), dtype=torch.uint8, device=device)
+        st = zero_state_t()
+        st.grad_dtype = grad_dtype
+        st.flags = flags
+        st.workspace = self.ws.data_ptr()
+        if stage in (1, 2):
+            part = zero_partition(N, Nd)
+            self.Np = part.Np
+            self.layer_len, self.layers, self.layer_padded = N, 1, [part.Np]
+            self.grads = [torch.zeros(N, dtype=gdt, device=device) for _ in range(Nd)]
+            self.params = [torch.zeros(N, dtype=torch.bfloat16, device=device)
+                           for _ in range(Nd)]
+            copies = 2 if flags == ZERO_FUSED else 1
+            self.master = [torch.zeros(self.Np, **f32) for _ in range(copies)]
+            self.exp_avg = [torch.zeros(self.Np, **f32) for _ in range(copies)]
+            self.exp_avg_sq = [torch.zeros(self.Np, **f32) for _ in range(copies)]
+            self.grad_shard = (torch.zeros(self.Np, **f32) if flags == ZERO_TWO_PASS else None)
+            self.param_shard = None
+        elif stage == 3:
+            L = layer_len if layer_len > 0 else N
+            self.layer_len = L
+            self.layers = (N + L - 1) // L if N > 0 else 0
+            self.layer_sizes = [min(L, N - l * L) for l in range(self.layers)]
+            self.layer_padded = [zero_partition(x, Nd).Np for x in self.layer_sizes]
+            self.Np = sum(self.layer_padded)
+            nbuf = N if per_layer_buffers else L
+            stride = L if per_layer_buffers else 0
+            self.grads = [torch.zeros(max(nbuf, 1), dtype=gdt, device=device) for _ in range(Nd)]
+            self.params = [torch.zeros(max(nbuf, 1), dtype=torch.bfloat16, device=device)
+                           for _ in range(Nd)]
+            self.master = [torch.zeros(self.Np, **f32)]
+            self.exp_avg = [torch.zeros(self.Np, **f32)]
+            self.exp_avg_sq = [torch.zeros(self.Np, **f32)]
+            self.grad_shard = torch.zeros(self.Np, **f32)
+            self.param_shard = torch.zeros(self.Np, dtype=torch.bfloat16, device=device)
+            st.grad_layer_stride = stride
+            st.param_layer_stride = stride
+        else:
+            raise ValueError("stage must be 1, 2 or 3")
+        for r in range(Nd):
+            st.grads[r] = self.grads[r].data_ptr()
+            st.params[r] = self.params[r].data_ptr()
+        for k in range(len(self.master)):
+            st.master[k] = self.master[k].data_ptr()
+            st.exp_avg[k] = self.exp_avg[k].data_ptr()
+            st.exp_avg_sq[k] = self.exp_avg_sq[k].data_ptr()
+        if self.grad_shard is not None:
+            st.grad_shard = self.grad_shard.data_ptr()
+        if self.param_shard is not None:
+            st.param_shard = self.param_shard.data_ptr()
+        self.state = st
+
+    def stream(self) -> int:
+        return self.torch.cuda.current_stream().cuda_stream
+
+    def init_workspace(self, t: int = 0) -> None:
+        zero_workspace_init(self.ws.data_ptr(), t, self.stream())
+
+    def step(self, hp: zero_hparams_t, bucket: int = 0) -> None:
+        b = bucket if self.stage in (1, 2) else self.layer_len
+        zero_step(self.stage, self.Nd, self.N, b, self.state, hp, self.stream())
+
+    def result(self) -> dict:
+        return zero_read_result(self.ws.data_ptr(), self.stream())
+
+    def live(self) -> int:
+        return self.result()["live"] if self.flags == ZERO_FUSED and self.stage in (1, 2) else 0
+
+    def sync_params_from_master(self) -> None:
+        """Write bf16(master) into every weight replica (stage 1/2) or the bf16 shards
+        (stage 3): the all-gather of the initial weights."""
+        live = self.live()
+        if self.stage in (1, 2):
+            zero_allgather(self.master[live].data_ptr(), [p.data_ptr() for p in self.params],
+                           self.Nd, 0, self.N, ZERO_GATE_ALWAYS, None, self.stream())
+        else:
+            zero_allgather(self.master[0].data_ptr(), [self.param_shard.data_ptr()], 1, 0,
+                           self.Np, ZERO_GATE_ALWAYS, None, self.stream())

@@ -1,0 +1,569 @@
+// zero_abi.cu -- host side of the C ABI declared in include/zero.h.
+//
+// Validates arguments, derives the element-independent scalars, sizes persistent grids to
+// the GPU, and enqueues the kernels of zero_kernels.cuh on the caller's stream.  It never
+// allocates memory and never synchronizes except in zero_read_result.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "zero.h"
+#include "zero_kernels.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(ZERO_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Resident CTAs per SM for each kernel, cached per device (occupancy does not change).
+constexpr int kMaxDevices = 64;
+enum KernelId {
+  kFusedBf16, kFusedFp16, kRsBf16, kRsFp16, kAdam, kCast, kGather, kNumKernels
+};
+
+const void* kernel_ptr(int id) {
+  switch (id) {
+    case kFusedBf16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0>);
+    case kFusedFp16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1>);
+    case kRsBf16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0>);
+    case kRsFp16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<1>);
+    case kAdam: return reinterpret_cast<const void*>(&zb::adam_kernel);
+    case kCast: return reinterpret_cast<const void*>(&zb::cast_allgather_kernel);
+    default: return reinterpret_cast<const void*>(&zb::gather_layer_kernel);
+  }
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int per_sm[kNumKernels] = {};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Persistent grid for `work` units of one thread each: at most one full wave of resident CTAs.
+int grid_for(int kid, int64_t work, int* grid) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(ZERO_EINVAL, "device ordinal %d unsupported", dev);
+  DeviceInfo& d = g_dev[dev];
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (d.sms == 0) {
+      e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    }
+    if (d.per_sm[kid] == 0) {
+      int n = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel_ptr(kid), zb::kThreads, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+      d.per_sm[kid] = n > 0 ? n : 1;
+    }
+  }
+  int64_t cap = (int64_t)d.sms * d.per_sm[kid];
+  if (cap > zb::kMaxCtas) cap = zb::kMaxCtas;
+  int64_t need = (work + zb::kThreads - 1) / zb::kThreads;
+  if (need < 1) need = 1;
+  *grid = (int)(need < cap ? need : cap);
+  return ZERO_OK;
+}
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ZERO_OK : cuda_fail(e, what);
+}
+
+zb::Header* header(void* ws) { return static_cast<zb::Header*>(ws); }
+zb::Partial* partials(void* ws) {
+  return reinterpret_cast<zb::Partial*>(static_cast<char*>(ws) + zb::kHeaderBytes);
+}
+
+int check_hp(const zero_hparams_t* hp) {
+  if (!hp) return fail(ZERO_EINVAL, "hparams is NULL");
+  if (!std::isfinite(hp->lr) || hp->lr < 0) return fail(ZERO_EINVAL, "lr must be finite and >= 0");
+  if (!(hp->beta1 >= 0 && hp->beta1 < 1)) return fail(ZERO_EINVAL, "beta1 must be in [0, 1)");
+  if (!(hp->beta2 >= 0 && hp->beta2 < 1)) return fail(ZERO_EINVAL, "beta2 must be in [0, 1)");
+  if (!(hp->eps > 0) || !std::isfinite(hp->eps)) return fail(ZERO_EINVAL, "eps must be finite and > 0");
+  if (!std::isfinite(hp->weight_decay)) return fail(ZERO_EINVAL, "weight_decay must be finite");
+  if (!(hp->loss_scale > 0) || !std::isfinite(hp->loss_scale))
+    return fail(ZERO_EINVAL, "loss_scale must be finite and > 0");
+  return ZERO_OK;
+}
+
+zb::Consts make_consts(const zero_hparams_t* hp, int Nd) {
+  zb::Consts c;
+  const double denom = hp->grad_average ? (double)Nd * hp->loss_scale : hp->loss_scale;
+  c.inv = (float)(1.0 / denom);
+  c.b1 = (float)hp->beta1;
+  c.b2 = (float)hp->beta2;
+  c.omb1 = (float)(1.0 - hp->beta1);
+  c.omb2 = (float)(1.0 - hp->beta2);
+  c.eps = (float)hp->eps;
+  c.decay = (float)(1.0 - hp->lr * hp->weight_decay);
+  c.unused = 0.0f;
+  c.lr = hp->lr;
+  c.b1d = hp->beta1;
+  c.b2d = hp->beta2;
+  return c;
+}
+
+int check_nd(int Nd) {
+  if (Nd < 1 || Nd > ZERO_MAX_ND) return fail(ZERO_EINVAL, "Nd=%d outside [1, %d]", Nd, ZERO_MAX_ND);
+  return ZERO_OK;
+}
+
+int check_window(int64_t lo, int64_t hi) {
+  if (lo < 0 || hi < lo) return fail(ZERO_EINVAL, "bad window [%lld, %lld)", (long long)lo, (long long)hi);
+  return ZERO_OK;
+}
+
+template <typename T>
+int check_ptrs(T* const* ptrs, int n, const char* what, bool* all_aligned) {
+  if (!ptrs) return fail(ZERO_EINVAL, "%s array is NULL", what);
+  for (int r = 0; r < n; ++r) {
+    if (!ptrs[r]) return fail(ZERO_EINVAL, "%s[%d] is NULL", what, r);
+    if (!aligned16(ptrs[r])) *all_aligned = false;
+  }
+  return ZERO_OK;
+}
+
+// Optional CUDA events recorded around the data-moving kernels of the next zero_step call
+// on this thread (one-shot; see zero_profile_events).
+thread_local cudaEvent_t g_prof_start = nullptr;
+thread_local cudaEvent_t g_prof_stop = nullptr;
+
+void prof_mark(bool start, cudaStream_t s) {
+  cudaEvent_t& e = start ? g_prof_start : g_prof_stop;
+  if (e) {
+    cudaEventRecord(e, s);
+    e = nullptr;
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+
+int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s) {
+  const int kid = dtype == ZERO_FP16 ? kFusedFp16 : kFusedBf16;
+  int grid = 0;
+  int rc = grid_for(kid, (a.hi - a.lo + 7) / 8, &grid);
+  if (rc) return rc;
+  if (dtype == ZERO_FP16)
+    zb::fused_step_kernel<1><<<grid, zb::kThreads, 0, s>>>(a);
+  else
+    zb::fused_step_kernel<0><<<grid, zb::kThreads, 0, s>>>(a);
+  return check_launch("fused_step_kernel launch");
+}
+
+int launch_rs(int dtype, const zb::RsArgs& a, cudaStream_t s) {
+  const int kid = dtype == ZERO_FP16 ? kRsFp16 : kRsBf16;
+  int grid = 0;
+  int rc = grid_for(kid, (a.hi - a.lo + 7) / 8, &grid);
+  if (rc) return rc;
+  if (dtype == ZERO_FP16)
+    zb::reduce_scatter_kernel<1><<<grid, zb::kThreads, 0, s>>>(a);
+  else
+    zb::reduce_scatter_kernel<0><<<grid, zb::kThreads, 0, s>>>(a);
+  return check_launch("reduce_scatter_kernel launch");
+}
+
+int launch_adam(const zb::AdamArgs& a, cudaStream_t s) {
+  int grid = 0;
+  int rc = grid_for(kAdam, (a.hi - a.lo + 7) / 8, &grid);
+  if (rc) return rc;
+  zb::adam_kernel<<<grid, zb::kThreads, 0, s>>>(a);
+  return check_launch("adam_kernel launch");
+}
+
+int launch_cast(const zb::CastArgs& a, cudaStream_t s) {
+  int grid = 0;
+  int rc = grid_for(kCast, (a.hi - a.lo + 7) / 8, &grid);
+  if (rc) return rc;
+  zb::cast_allgather_kernel<<<grid, zb::kThreads, 0, s>>>(a);
+  return check_launch("cast_allgather_kernel launch");
+}
+
+int launch_ws(void* ws, int op, long long t0, cudaStream_t s) {
+  zb::ws_ctl_kernel<<<1, 32, 0, s>>>(header(ws), op, t0);
+  return check_launch("ws_ctl_kernel launch");
+}
+
+int do_gather(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* const* out, int nout,
+              cudaStream_t s) {
+  if (L == 0) return ZERO_OK;
+  zb::GatherArgs a;
+  std::memset(&a, 0, sizeof a);
+  bool al = true;
+  int rc = check_ptrs(shards, Nd, "shards", &al);
+  if (rc) return rc;
+  rc = check_ptrs(out, nout, "out", &al);
+  if (rc) return rc;
+  const int64_t S = (L + Nd - 1) / Nd;
+  for (int r = 0; r < Nd; ++r) a.shards[r] = shards[r];
+  for (int o = 0; o < nout; ++o) a.out[o] = out[o];
+  a.Nd = Nd;
+  a.nout = nout;
+  a.L = L;
+  a.S = S;
+  a.vec = al && (S % 8 == 0);
+  int grid = 0;
+  rc = grid_for(kGather, (S + 7) / 8, &grid);
+  if (rc) return rc;
+  int gx = (grid + Nd - 1) / Nd;  // keep about one wave in total over the Nd rows
+  if (gx < 1) gx = 1;
+  zb::gather_layer_kernel<<<dim3(gx, Nd), zb::kThreads, 0, s>>>(a);
+  return check_launch("gather_layer_kernel launch");
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+const char* zero_last_error(void) { return g_err; }
+
+const char* zero_version(void) { return "zero-b200 1.0 sm_100a"; }
+
+int zero_partition(int64_t N, int Nd, zero_partition_t* out) {
+  if (!out) return fail(ZERO_EINVAL, "out is NULL");
+  if (N < 0) return fail(ZERO_EINVAL, "N=%lld < 0", (long long)N);
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  const int64_t S = (N + Nd - 1) / Nd;
+  out->N = N;
+  out->Nd = Nd;
+  out->reserved = 0;
+  out->S = S;
+  out->Np = S * Nd;
+  out->pad = S * Nd - N;
+  return ZERO_OK;
+}
+
+size_t zero_workspace_bytes(void) { return zb::kWorkspaceBytes; }
+
+int zero_workspace_init(void* ws, int64_t t, void* stream) {
+  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (t < 0) return fail(ZERO_EINVAL, "t=%lld < 0", (long long)t);
+  return launch_ws(ws, zb::kWsInit, t, (cudaStream_t)stream);
+}
+
+int zero_read_result(const void* ws, zero_step_result_t* out, void* stream) {
+  if (!ws || !out) return fail(ZERO_EINVAL, "workspace or out is NULL");
+  zb::Header h;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof h, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(result)");
+  e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  out->step = h.t;
+  out->skipped = h.skipped;
+  out->overflow = h.last_flag;
+  out->live = h.live;
+  out->grad_sumsq = h.last_sumsq;
+  out->pending_overflow = h.pending_flag;
+  out->reserved = 0;
+  out->pending_sumsq = h.pending_sumsq;
+  return ZERO_OK;
+}
+
+int zero_profile_events(void* start_event, void* stop_event) {
+  g_prof_start = (cudaEvent_t)start_event;
+  g_prof_stop = (cudaEvent_t)stop_event;
+  return ZERO_OK;
+}
+
+int zero_begin_step(void* ws, void* stream) {
+  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  return launch_ws(ws, zb::kWsBegin, 0, (cudaStream_t)stream);
+}
+
+int zero_end_step(void* ws, void* stream) {
+  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  return launch_ws(ws, zb::kWsEnd, 0, (cudaStream_t)stream);
+}
+
+int zero_reduce_scatter(const uint16_t* const* grads, int dtype, int Nd, int64_t lo, int64_t hi,
+                        const zero_hparams_t* hp, float* grad_out, void* ws, void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if ((rc = check_window(lo, hi))) return rc;
+  if ((rc = check_hp(hp))) return rc;
+  if (dtype != ZERO_BF16 && dtype != ZERO_FP16) return fail(ZERO_EINVAL, "dtype=%d", dtype);
+  if (!grad_out || !ws) return fail(ZERO_EINVAL, "grad_out or workspace is NULL");
+  zb::RsArgs a;
+  std::memset(&a, 0, sizeof a);
+  bool al = aligned16(grad_out);
+  if ((rc = check_ptrs(grads, Nd, "grads", &al))) return rc;
+  for (int r = 0; r < Nd; ++r) a.grads[r] = grads[r];
+  a.out = grad_out;
+  a.lo = lo;
+  a.hi = hi;
+  a.inv = make_consts(hp, Nd).inv;
+  a.Nd = Nd;
+  a.hdr = header(ws);
+  a.part = partials(ws);
+  a.mode = zb::kAccAdd;
+  a.vec = al;
+  return launch_rs(dtype, a, (cudaStream_t)stream);
+}
+
+int zero_adam_shard(float* master, float* exp_avg, float* exp_avg_sq, const float* grad, int64_t lo,
+                    int64_t hi, const zero_hparams_t* hp, uint16_t* param_out, void* ws, void* stream) {
+  int rc = check_window(lo, hi);
+  if (rc) return rc;
+  if ((rc = check_hp(hp))) return rc;
+  if (!master || !exp_avg || !exp_avg_sq || !grad || !ws)
+    return fail(ZERO_EINVAL, "master, exp_avg, exp_avg_sq, grad and workspace must be non-NULL");
+  zb::AdamArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.p[0] = a.p[1] = master;
+  a.m[0] = a.m[1] = exp_avg;
+  a.v[0] = a.v[1] = exp_avg_sq;
+  a.g = grad;
+  a.out16 = param_out;
+  a.nrep = 0;
+  a.use_live = 0;
+  a.lo = lo;
+  a.hi = hi;
+  a.c = make_consts(hp, 1);
+  a.hdr = header(ws);
+  a.part = partials(ws);
+  a.mode = 0;
+  a.vec = aligned16(master) && aligned16(exp_avg) && aligned16(exp_avg_sq) && aligned16(grad) &&
+          (param_out == nullptr || aligned16(param_out));
+  return launch_adam(a, (cudaStream_t)stream);
+}
+
+int zero_allgather(const float* master, uint16_t* const* replicas, int Nd, int64_t lo, int64_t hi, int gate,
+                   const void* ws, void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if ((rc = check_window(lo, hi))) return rc;
+  if (!master) return fail(ZERO_EINVAL, "master is NULL");
+  if (gate != ZERO_GATE_ALWAYS && gate != ZERO_GATE_NO_OVERFLOW) return fail(ZERO_EINVAL, "gate=%d", gate);
+  if (gate == ZERO_GATE_NO_OVERFLOW && !ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  zb::CastArgs a;
+  std::memset(&a, 0, sizeof a);
+  bool al = aligned16(master);
+  if ((rc = check_ptrs(replicas, Nd, "replicas", &al))) return rc;
+  a.src[0] = a.src[1] = master;
+  for (int r = 0; r < Nd; ++r) a.reps[r] = replicas[r];
+  a.nrep = Nd;
+  a.gate = gate == ZERO_GATE_NO_OVERFLOW ? zb::kGateNoOverflow : zb::kGateAlways;
+  a.lo = lo;
+  a.hi = hi;
+  a.hdr = static_cast<const zb::Header*>(ws);
+  a.vec = al;
+  return launch_cast(a, (cudaStream_t)stream);
+}
+
+int zero3_gather_layer(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* const* out, int nout,
+                       void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if (nout < 1 || nout > ZERO_MAX_ND) return fail(ZERO_EINVAL, "nout=%d outside [1, %d]", nout, ZERO_MAX_ND);
+  if (L < 0) return fail(ZERO_EINVAL, "L=%lld < 0", (long long)L);
+  return do_gather(shards, Nd, L, out, nout, (cudaStream_t)stream);
+}
+
+int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* st, const zero_hparams_t* hp,
+              void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if ((rc = check_hp(hp))) return rc;
+  if (!st) return fail(ZERO_EINVAL, "state is NULL");
+  if (stage < 1 || stage > 3) return fail(ZERO_EINVAL, "stage=%d outside [1, 3]", stage);
+  if (N < 0 || bucket < 0) return fail(ZERO_EINVAL, "N and bucket must be >= 0");
+  if (st->grad_dtype != ZERO_BF16 && st->grad_dtype != ZERO_FP16)
+    return fail(ZERO_EINVAL, "grad_dtype=%d", st->grad_dtype);
+  if (!st->workspace) return fail(ZERO_EINVAL, "workspace is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  const zb::Consts c = make_consts(hp, Nd);
+  void* ws = st->workspace;
+  if (N == 0) {  // nothing to reduce or update: the (empty) step completes without overflow
+    prof_mark(true, s);
+    prof_mark(false, s);
+    return launch_ws(ws, zb::kWsEnd, 0, s);
+  }
+
+  if (stage == 3) {
+    if (!st->master[0] || !st->exp_avg[0] || !st->exp_avg_sq[0] || !st->grad_shard || !st->param_shard)
+      return fail(ZERO_EINVAL, "stage 3 needs master[0], exp_avg[0], exp_avg_sq[0], grad_shard, param_shard");
+    bool al = true;
+    if ((rc = check_ptrs(st->grads, Nd, "grads", &al))) return rc;
+    if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
+    const int64_t L = bucket > 0 ? bucket : N;
+    const int64_t nl = (N + L - 1) / L;
+    prof_mark(true, s);
+    int64_t off = 0;
+    for (int64_t l = 0; l < nl; ++l) {  // forward gathers + backward reduce-scatters, layer by layer
+      const int64_t Ll = (l + 1) * L <= N ? L : N - l * L;
+      const int64_t Sl = (Ll + Nd - 1) / Nd;
+      const uint16_t* shards[ZERO_MAX_ND];
+      uint16_t* outs[ZERO_MAX_ND];
+      const uint16_t* gl[ZERO_MAX_ND];
+      for (int r = 0; r < Nd; ++r) {
+        shards[r] = st->param_shard + off + r * Sl;
+        outs[r] = st->params[r] + l * st->param_layer_stride;
+        gl[r] = st->grads[r] + l * st->grad_layer_stride;
+      }
+      if ((rc = do_gather(shards, Nd, Ll, outs, Nd, s))) return rc;
+      zb::RsArgs a;
+      std::memset(&a, 0, sizeof a);
+      bool ral = aligned16(st->grad_shard + off);
+      for (int r = 0; r < Nd; ++r) {
+        a.grads[r] = gl[r];
+        ral = ral && aligned16(gl[r]);
+      }
+      a.out = st->grad_shard + off;
+      a.lo = 0;
+      a.hi = Ll;
+      a.inv = c.inv;
+      a.Nd = Nd;
+      a.hdr = header(ws);
+      a.part = partials(ws);
+      a.mode = l == 0 ? zb::kAccSet : zb::kAccAdd;
+      a.vec = ral;
+      if ((rc = launch_rs(st->grad_dtype, a, s))) return rc;
+      off += Sl * Nd;
+    }
+    off = 0;
+    for (int64_t l = 0; l < nl; ++l) {  // optimizer step on every shard, gated on the overflow flag
+      const int64_t Ll = (l + 1) * L <= N ? L : N - l * L;
+      const int64_t Sl = (Ll + Nd - 1) / Nd;
+      zb::AdamArgs a;
+      std::memset(&a, 0, sizeof a);
+      a.p[0] = a.p[1] = st->master[0] + off;
+      a.m[0] = a.m[1] = st->exp_avg[0] + off;
+      a.v[0] = a.v[1] = st->exp_avg_sq[0] + off;
+      a.g = st->grad_shard + off;
+      a.out16 = st->param_shard + off;
+      a.lo = 0;
+      a.hi = Ll;
+      a.c = c;
+      a.hdr = header(ws);
+      a.part = partials(ws);
+      a.mode = l == nl - 1 ? zb::kFinalize : 0;
+      a.vec = aligned16(a.p[0]) && aligned16(a.m[0]) && aligned16(a.v[0]) && aligned16(a.g) &&
+              aligned16(a.out16);
+      if ((rc = launch_adam(a, s))) return rc;
+      off += Sl * Nd;
+    }
+    prof_mark(false, s);
+    return ZERO_OK;
+  }
+
+  // stages 1 and 2
+  bool al = true;
+  if ((rc = check_ptrs(st->grads, Nd, "grads", &al))) return rc;
+  if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
+  const int64_t B = bucket > 0 ? bucket : N;
+  const int64_t nb = (N + B - 1) / B;
+
+  if (st->flags & ZERO_TWO_PASS) {
+    if (!st->master[0] || !st->exp_avg[0] || !st->exp_avg_sq[0] || !st->grad_shard)
+      return fail(ZERO_EINVAL, "ZERO_TWO_PASS needs master[0], exp_avg[0], exp_avg_sq[0], grad_shard");
+    prof_mark(true, s);
+    for (int64_t k = 0; k < nb; ++k) {
+      zb::RsArgs a;
+      std::memset(&a, 0, sizeof a);
+      for (int r = 0; r < Nd; ++r) a.grads[r] = st->grads[r];
+      a.out = st->grad_shard;
+      a.lo = k * B;
+      a.hi = (k + 1) * B < N ? (k + 1) * B : N;
+      a.inv = c.inv;
+      a.Nd = Nd;
+      a.hdr = header(ws);
+      a.part = partials(ws);
+      a.mode = k == 0 ? zb::kAccSet : zb::kAccAdd;
+      a.vec = al && aligned16(st->grad_shard);
+      if ((rc = launch_rs(st->grad_dtype, a, s))) return rc;
+    }
+    // copy 1 may be absent on this path; `live` then must be 0
+    const bool two = st->master[1] && st->exp_avg[1] && st->exp_avg_sq[1];
+    for (int64_t k = 0; k < nb; ++k) {
+      zb::AdamArgs a;
+      std::memset(&a, 0, sizeof a);
+      for (int i = 0; i < 2; ++i) {
+        a.p[i] = two ? st->master[i] : st->master[0];
+        a.m[i] = two ? st->exp_avg[i] : st->exp_avg[0];
+        a.v[i] = two ? st->exp_avg_sq[i] : st->exp_avg_sq[0];
+      }
+      a.g = st->grad_shard;
+      for (int r = 0; r < Nd; ++r) a.reps[r] = st->params[r];
+      a.nrep = Nd;
+      a.use_live = 1;
+      a.lo = k * B;
+      a.hi = (k + 1) * B < N ? (k + 1) * B : N;
+      a.c = c;
+      a.hdr = header(ws);
+      a.part = partials(ws);
+      a.mode = k == nb - 1 ? zb::kFinalize : 0;
+      a.vec = al && aligned16(a.p[0]) && aligned16(a.p[1]) && aligned16(a.m[0]) && aligned16(a.m[1]) &&
+              aligned16(a.v[0]) && aligned16(a.v[1]) && aligned16(a.g);
+      if ((rc = launch_adam(a, s))) return rc;
+    }
+    prof_mark(false, s);
+    return ZERO_OK;
+  }
+
+  for (int i = 0; i < 2; ++i)
+    if (!st->master[i] || !st->exp_avg[i] || !st->exp_avg_sq[i])
+      return fail(ZERO_EINVAL, "ZERO_FUSED needs both state copies (master/exp_avg/exp_avg_sq [0] and [1])");
+  zb::FusedArgs a;
+  std::memset(&a, 0, sizeof a);
+  for (int r = 0; r < Nd; ++r) {
+    a.grads[r] = st->grads[r];
+    a.reps[r] = st->params[r];
+  }
+  for (int i = 0; i < 2; ++i) {
+    a.p[i] = st->master[i];
+    a.m[i] = st->exp_avg[i];
+    a.v[i] = st->exp_avg_sq[i];
+    al = al && aligned16(a.p[i]) && aligned16(a.m[i]) && aligned16(a.v[i]);
+  }
+  a.c = c;
+  a.hdr = header(ws);
+  a.part = partials(ws);
+  a.Nd = Nd;
+  a.vec = al;
+  prof_mark(true, s);
+  for (int64_t k = 0; k < nb; ++k) {
+    a.lo = k * B < N ? k * B : N;
+    a.hi = (k + 1) * B < N ? (k + 1) * B : N;
+    a.mode = (k == 0 ? zb::kAccSet : zb::kAccAdd) | (k == nb - 1 ? (zb::kFinalize | zb::kFlip) : 0);
+    if ((rc = launch_fused(st->grad_dtype, a, s))) return rc;
+  }
+  prof_mark(false, s);
+  // overflow repair: rewrite the replicas from the unchanged state (runs only after a skip)
+  zb::CastArgs r;
+  std::memset(&r, 0, sizeof r);
+  r.src[0] = st->master[0];
+  r.src[1] = st->master[1];
+  for (int q = 0; q < Nd; ++q) r.reps[q] = st->params[q];
+  r.nrep = Nd;
+  r.gate = zb::kGateRepair;
+  r.lo = 0;
+  r.hi = N;
+  r.hdr = header(ws);
+  r.vec = al;
+  return launch_cast(r, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,629 @@
+// zero_kernels.cuh -- sm_100a kernels of the sharded mixed-precision Adam step (ZeRO-1/2/3).
+//
+// Every kernel here streams HBM: per element it does a few dozen fp32 operations against
+// tens of bytes of traffic (about 0.35 flop/byte), far below the ridge point, so there are
+// no tensor-core paths.  The design choices are the ones that matter for a bandwidth-bound
+// kernel on B200: 16-byte vector loads/stores with streaming cache hints, an Nd-way fan-in
+// issued as independent loads in flight per thread, persistent grids sized to a multiple of
+// the 148 SMs, and a single pass over the data wherever the algorithm allows.
+//
+// Simulated collectives ([P1] §二 and §三, [P3] core operations; page titles in include/zero.h):
+// the Nd "ranks" are Nd buffers in this GPU's memory.  A reduce-scatter is the Nd-way read of
+// the gradient replicas at an index (each index belongs to exactly one rank's shard), an
+// all-gather is the Nd-way write of the bf16 weight at that index.  Because both act on the
+// same index as the Adam update, the fused kernel does RS + Adam + AG in one pass.
+//
+// Numerics: every fp32 operation is an explicit round-to-nearest intrinsic (no contraction),
+// replicas are summed in rank order, and the per-element rule is the one documented for
+// zero_adam_shard in include/zero.h.  The overflow flag is an OR (exact), the sum of squares
+// is accumulated in double in a fixed order for a given grid.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace zb {
+
+constexpr int kMaxNd = 64;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxCtas = 8192;
+
+// Step bookkeeping at the start of the workspace.
+struct Header {
+  unsigned int done;      // CTAs of the current launch that have finished (reset by the last one)
+  int pending_flag;       // overflow seen by the step in progress
+  double pending_sumsq;   // sum of squares accumulated by the step in progress
+  long long t;            // completed updates
+  long long skipped;      // skipped steps
+  int live;               // state copy holding the current state (fused path)
+  int last_flag;          // overflow of the last finished step
+  double last_sumsq;      // sum of squares of the last finished step
+};
+static_assert(sizeof(Header) <= 256, "header must fit its slot");
+
+struct Partial {
+  double sumsq;
+  int flag;
+  int pad;
+};
+
+constexpr size_t kHeaderBytes = 256;
+constexpr size_t kWorkspaceBytes = kHeaderBytes + sizeof(Partial) * kMaxCtas;
+
+// What the last CTA of a launch does with the launch's totals.
+enum : int {
+  kAccSet = 1,    // pending := launch totals (first launch of a step)
+  kAccAdd = 2,    // pending += launch totals
+  kFinalize = 4,  // end the step: t += 1 unless overflow (else skipped += 1)
+  kFlip = 8,      // with kFinalize and no overflow: swap the live state copy
+};
+
+// Element-independent scalars, rounded once to fp32 on the host (see include/zero.h).
+struct Consts {
+  float inv;    // 1/(Nd*loss_scale) or 1/loss_scale
+  float b1, b2;
+  float omb1, omb2;
+  float eps;
+  float decay;  // 1 - lr*wd
+  float unused;
+  double lr, b1d, b2d;  // for the step-dependent bias corrections
+};
+
+struct Bias {
+  float step_size;  // lr / (1 - b1^t)
+  float sbc2;       // sqrt(1 - b2^t)
+};
+
+// b^e for e >= 0 by binary exponentiation (square-and-multiply, Knuth TAOCP vol. 2, 4.6.3),
+// every product one double round-to-nearest step.
+__device__ __forceinline__ double pow_binary(double b, long long e) {
+  double r = 1.0;
+  while (e > 0) {
+    if (e & 1) r = __dmul_rn(r, b);
+    b = __dmul_rn(b, b);
+    e >>= 1;
+  }
+  return r;
+}
+
+__device__ __forceinline__ Bias bias_for(const Consts& c, long long t) {
+  Bias o;
+  o.step_size = __double2float_rn(__ddiv_rn(c.lr, __dadd_rn(1.0, -pow_binary(c.b1d, t))));
+  o.sbc2 = __double2float_rn(__dsqrt_rn(__dadd_rn(1.0, -pow_binary(c.b2d, t))));
+  return o;
+}
+
+// One Adam/AdamW update of one element (the rule of zero_adam_shard).  With wd = 0 the decay
+// factor is exactly 1 and the first multiply changes nothing.
+__device__ __forceinline__ void adam_elem(float g, float& p, float& m, float& v, const Consts& c,
+                                          const Bias& b) {
+  p = __fmul_rn(p, c.decay);
+  m = __fadd_rn(__fmul_rn(c.b1, m), __fmul_rn(c.omb1, g));
+  v = __fadd_rn(__fmul_rn(c.b2, v), __fmul_rn(__fmul_rn(c.omb2, g), g));
+  const float den = __fadd_rn(__fdiv_rn(__fsqrt_rn(v), b.sbc2), c.eps);
+  p = __fsub_rn(p, __fmul_rn(b.step_size, __fdiv_rn(m, den)));
+}
+
+__device__ __forceinline__ int nonfinite(float x) {
+  return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
+}
+
+// ------------------------------------------------------------------ memory helpers
+
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ float4 ld_stream(const float* p) {
+  return __ldcs(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ void st_stream(uint16_t* p, uint4 v) {
+  __stcs(reinterpret_cast<uint4*>(p), v);
+}
+__device__ __forceinline__ void st_stream(float* p, float4 v) {
+  __stcs(reinterpret_cast<float4*>(p), v);
+}
+
+// 16-bit gradient decoding (exact).
+template <int DT>
+struct Dec;
+
+template <>
+struct Dec<0> {  // bf16: the upper half of an fp32 word
+  __device__ static __forceinline__ float one(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+  __device__ static __forceinline__ void add2(float& a, float& b, uint32_t w) {
+    a = __fadd_rn(a, __uint_as_float(w << 16));
+    b = __fadd_rn(b, __uint_as_float(w & 0xffff0000u));
+  }
+};
+
+template <>
+struct Dec<1> {  // IEEE fp16
+  __device__ static __forceinline__ float one(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+  __device__ static __forceinline__ void add2(float& a, float& b, uint32_t w) {
+    __half2 h2;
+    *reinterpret_cast<uint32_t*>(&h2) = w;
+    const float2 f = __half22float2(h2);
+    a = __fadd_rn(a, f.x);
+    b = __fadd_rn(b, f.y);
+  }
+};
+
+template <int DT>
+__device__ __forceinline__ void add8(float (&s)[8], const uint4& q) {
+  Dec<DT>::add2(s[0], s[1], q.x);
+  Dec<DT>::add2(s[2], s[3], q.y);
+  Dec<DT>::add2(s[4], s[5], q.z);
+  Dec<DT>::add2(s[6], s[7], q.w);
+}
+
+// Rank-order sum of the Nd replicas at 8 consecutive elements starting at i (16-byte aligned).
+// Loads are issued 8 ranks at a time so that up to 128 bytes per thread are in flight.
+template <int DT>
+__device__ __forceinline__ void fan_in8(const uint16_t* const* grads, int Nd, int64_t i, float (&s)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) s[k] = 0.0f;
+  for (int r0 = 0; r0 < Nd; r0 += 8) {
+    uint4 q[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (r0 + u < Nd) q[u] = ld_stream(grads[r0 + u] + i);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (r0 + u < Nd) add8<DT>(s, q[u]);
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ float fan_in1(const uint16_t* const* grads, int Nd, int64_t i) {
+  float s = 0.0f;
+  for (int r = 0; r < Nd; ++r) s = __fadd_rn(s, Dec<DT>::one(grads[r][i]));
+  return s;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo, round to nearest even
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&p)[8]) {
+  return make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                    pack_bf16x2(p[6], p[7]));
+}
+
+__device__ __forceinline__ uint16_t to_bf16(float x) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return *reinterpret_cast<const uint16_t*>(&h);
+}
+
+__device__ __forceinline__ void unpack(const float4& a, const float4& b, float (&x)[8]) {
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// Vector bounds of a window: the 8-aligned interior [vlo, vhi) and the scalar remainder.
+struct Span {
+  int64_t vlo, vhi, nvec, nhead, nrest;
+  __device__ __forceinline__ Span(int64_t lo, int64_t hi, int vec) {
+    vlo = lo;
+    vhi = lo;
+    if (vec) {
+      vlo = (lo + 7) & ~int64_t(7);
+      if (vlo > hi) vlo = hi;
+      vhi = hi & ~int64_t(7);
+      if (vhi < vlo) vhi = vlo;
+    }
+    nvec = (vhi - vlo) >> 3;
+    nhead = vlo - lo;
+    nrest = nhead + (hi - vhi);
+  }
+  // e-th scalar element: the head [lo, vlo) then the tail [vhi, hi)
+  __device__ __forceinline__ int64_t scalar_index(int64_t lo, int64_t e) const {
+    return e < nhead ? lo + e : vhi + (e - nhead);
+  }
+};
+
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = __dadd_rn(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// Launch epilogue: per-CTA totals into the partials, and the last CTA to arrive reduces them
+// in CTA order and applies `mode` to the header.  No CTA waits for another (the last one to
+// arrive does the work), so there is no spin and no co-residency assumption.
+__device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Partial* part, int mode) {
+  if (mode == 0) return;
+  __shared__ double r_sq[kWarps];
+  __shared__ int r_bad[kWarps];
+  __shared__ int am_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  sq = warp_sum(sq);
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    r_sq[warp] = sq;
+    r_bad[warp] = bad;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    int f = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      s = __dadd_rn(s, r_sq[w]);
+      f |= r_bad[w];
+    }
+    part[blockIdx.x].sumsq = s;
+    part[blockIdx.x].flag = f;
+    __threadfence();
+    const unsigned prev = atomicAdd(&hdr->done, 1u);
+    am_last = (prev == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!am_last) return;
+  __threadfence();
+  double s = 0.0;
+  int f = 0;
+  for (int k = threadIdx.x; k < (int)gridDim.x; k += kThreads) {
+    s = __dadd_rn(s, __ldcg(&part[k].sumsq));
+    f |= __ldcg(&part[k].flag);
+  }
+  s = warp_sum(s);
+  f = __any_sync(0xffffffffu, f);
+  __syncthreads();
+  if (lane == 0) {
+    r_sq[warp] = s;
+    r_bad[warp] = f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    int fl = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      tot = __dadd_rn(tot, r_sq[w]);
+      fl |= r_bad[w];
+    }
+    if (mode & kAccSet) {
+      hdr->pending_flag = fl;
+      hdr->pending_sumsq = tot;
+    } else if (mode & kAccAdd) {
+      hdr->pending_flag |= fl;
+      hdr->pending_sumsq = __dadd_rn(hdr->pending_sumsq, tot);
+    }
+    if (mode & kFinalize) {
+      const int of = hdr->pending_flag;
+      hdr->last_flag = of;
+      hdr->last_sumsq = hdr->pending_sumsq;
+      if (!of) {
+        hdr->t += 1;
+        if (mode & kFlip) hdr->live ^= 1;
+      } else {
+        hdr->skipped += 1;
+      }
+      hdr->pending_flag = 0;
+      hdr->pending_sumsq = 0.0;
+    }
+    hdr->done = 0u;
+    __threadfence();
+  }
+}
+
+// ------------------------------------------------------------------ K1: fused RS + Adam + AG
+
+struct FusedArgs {
+  const uint16_t* grads[kMaxNd];  // Nd gradient replicas
+  uint16_t* reps[kMaxNd];         // Nd bf16 weight replicas
+  float* p[2];                    // master weights, two copies (read live, write 1-live)
+  float* m[2];
+  float* v[2];
+  int64_t lo, hi;                 // window of global indices
+  Consts c;
+  Header* hdr;
+  Partial* part;
+  int Nd;
+  int mode;
+  int vec;
+  int unused;
+};
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_constant__ FusedArgs a) {
+  __shared__ Bias s_bias;
+  __shared__ int s_live;
+  if (threadIdx.x == 0) {
+    s_bias = bias_for(a.c, __ldcg(&a.hdr->t) + 1);
+    s_live = __ldcg(&a.hdr->live) & 1;
+  }
+  __syncthreads();
+  const Bias b = s_bias;
+  const int live = s_live;
+  const float* __restrict__ sp = a.p[live];
+  const float* __restrict__ sm = a.m[live];
+  const float* __restrict__ sv = a.v[live];
+  float* __restrict__ dp = a.p[live ^ 1];
+  float* __restrict__ dm = a.m[live ^ 1];
+  float* __restrict__ dv = a.v[live ^ 1];
+
+  double sq = 0.0;
+  int bad = 0;
+  const Span sp8(a.lo, a.hi, a.vec);
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < sp8.nvec; j += stride) {
+    const int64_t i = sp8.vlo + (j << 3);
+    float P[8], M[8], V[8], s[8];
+    unpack(ld_stream(sp + i), ld_stream(sp + i + 4), P);
+    unpack(ld_stream(sm + i), ld_stream(sm + i + 4), M);
+    unpack(ld_stream(sv + i), ld_stream(sv + i + 4), V);
+    fan_in8<DT>(a.grads, a.Nd, i, s);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float g = __fmul_rn(s[k], a.c.inv);
+      bad |= nonfinite(g);
+      sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
+      adam_elem(g, P[k], M[k], V[k], a.c, b);
+    }
+    st_stream(dp + i, make_float4(P[0], P[1], P[2], P[3]));
+    st_stream(dp + i + 4, make_float4(P[4], P[5], P[6], P[7]));
+    st_stream(dm + i, make_float4(M[0], M[1], M[2], M[3]));
+    st_stream(dm + i + 4, make_float4(M[4], M[5], M[6], M[7]));
+    st_stream(dv + i, make_float4(V[0], V[1], V[2], V[3]));
+    st_stream(dv + i + 4, make_float4(V[4], V[5], V[6], V[7]));
+    const uint4 w = pack_bf16x8(P);
+    for (int r = 0; r < a.Nd; ++r) st_stream(a.reps[r] + i, w);
+  }
+  for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
+    const int64_t i = sp8.scalar_index(a.lo, e);
+    const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), a.c.inv);
+    bad |= nonfinite(g);
+    sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
+    float P = sp[i], M = sm[i], V = sv[i];
+    adam_elem(g, P, M, V, a.c, b);
+    dp[i] = P;
+    dm[i] = M;
+    dv[i] = V;
+    const uint16_t w = to_bf16(P);
+    for (int r = 0; r < a.Nd; ++r) a.reps[r][i] = w;
+  }
+  block_finish(sq, bad, a.hdr, a.part, a.mode);
+}
+
+// ------------------------------------------------------------------ K3: RS into an fp32 shard
+
+struct RsArgs {
+  const uint16_t* grads[kMaxNd];
+  float* out;        // reduced gradient, indexed like the replicas
+  int64_t lo, hi;
+  float inv;
+  int Nd;
+  Header* hdr;
+  Partial* part;
+  int mode;
+  int vec;
+};
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_constant__ RsArgs a) {
+  double sq = 0.0;
+  int bad = 0;
+  float* __restrict__ out = a.out;
+  const Span sp8(a.lo, a.hi, a.vec);
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < sp8.nvec; j += stride) {
+    const int64_t i = sp8.vlo + (j << 3);
+    float s[8];
+    fan_in8<DT>(a.grads, a.Nd, i, s);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      s[k] = __fmul_rn(s[k], a.inv);
+      bad |= nonfinite(s[k]);
+      sq = __dadd_rn(sq, __dmul_rn((double)s[k], (double)s[k]));
+    }
+    st_stream(out + i, make_float4(s[0], s[1], s[2], s[3]));
+    st_stream(out + i + 4, make_float4(s[4], s[5], s[6], s[7]));
+  }
+  for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
+    const int64_t i = sp8.scalar_index(a.lo, e);
+    const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), a.inv);
+    bad |= nonfinite(g);
+    sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
+    out[i] = g;
+  }
+  block_finish(sq, bad, a.hdr, a.part, a.mode);
+}
+
+// ------------------------------------------------------------------ K4: gated Adam (+ cast / AG)
+
+struct AdamArgs {
+  float* p[2];        // state copies; the kernel updates copy `live` in place
+  float* m[2];
+  float* v[2];
+  const float* g;     // reduced gradient
+  uint16_t* out16;    // optional bf16 copy of the new weights (ZeRO-3 shard)
+  uint16_t* reps[kMaxNd];  // optional bf16 replicas (fused all-gather of the two-pass path)
+  int nrep;
+  int use_live;       // 0: always copy 0
+  int64_t lo, hi;
+  Consts c;
+  Header* hdr;
+  Partial* part;
+  int mode;
+  int vec;
+};
+
+__global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ AdamArgs a) {
+  __shared__ Bias s_bias;
+  __shared__ int s_live, s_skip;
+  if (threadIdx.x == 0) {
+    s_bias = bias_for(a.c, __ldcg(&a.hdr->t) + 1);
+    s_live = a.use_live ? (__ldcg(&a.hdr->live) & 1) : 0;
+    s_skip = __ldcg(&a.hdr->pending_flag);
+  }
+  __syncthreads();
+  if (!s_skip) {
+    const Bias b = s_bias;
+    float* __restrict__ P_ = a.p[s_live];
+    float* __restrict__ M_ = a.m[s_live];
+    float* __restrict__ V_ = a.v[s_live];
+    const float* __restrict__ G_ = a.g;
+    const Span sp8(a.lo, a.hi, a.vec);
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < sp8.nvec; j += stride) {
+      const int64_t i = sp8.vlo + (j << 3);
+      float P[8], M[8], V[8], G[8];
+      unpack(ld_stream(P_ + i), ld_stream(P_ + i + 4), P);
+      unpack(ld_stream(M_ + i), ld_stream(M_ + i + 4), M);
+      unpack(ld_stream(V_ + i), ld_stream(V_ + i + 4), V);
+      unpack(ld_stream(G_ + i), ld_stream(G_ + i + 4), G);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) adam_elem(G[k], P[k], M[k], V[k], a.c, b);
+      st_stream(P_ + i, make_float4(P[0], P[1], P[2], P[3]));
+      st_stream(P_ + i + 4, make_float4(P[4], P[5], P[6], P[7]));
+      st_stream(M_ + i, make_float4(M[0], M[1], M[2], M[3]));
+      st_stream(M_ + i + 4, make_float4(M[4], M[5], M[6], M[7]));
+      st_stream(V_ + i, make_float4(V[0], V[1], V[2], V[3]));
+      st_stream(V_ + i + 4, make_float4(V[4], V[5], V[6], V[7]));
+      if (a.out16 || a.nrep) {
+        const uint4 w = pack_bf16x8(P);
+        if (a.out16) st_stream(a.out16 + i, w);
+        for (int r = 0; r < a.nrep; ++r) st_stream(a.reps[r] + i, w);
+      }
+    }
+    for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
+      const int64_t i = sp8.scalar_index(a.lo, e);
+      float P = P_[i], M = M_[i], V = V_[i];
+      adam_elem(G_[i], P, M, V, a.c, b);
+      P_[i] = P;
+      M_[i] = M;
+      V_[i] = V;
+      const uint16_t w = to_bf16(P);
+      if (a.out16) a.out16[i] = w;
+      for (int r = 0; r < a.nrep; ++r) a.reps[r][i] = w;
+    }
+  }
+  block_finish(0.0, 0, a.hdr, a.part, a.mode);
+}
+
+// ------------------------------------------------------------------ K5: cast + all-gather
+
+enum : int {
+  kGateAlways = 0,
+  kGateNoOverflow = 1,  // skip if the step in progress has overflowed
+  kGateRepair = 2,      // run only if the last finished step overflowed; source = copy `live`
+};
+
+struct CastArgs {
+  const float* src[2];
+  uint16_t* reps[kMaxNd];
+  int nrep;
+  int gate;
+  int64_t lo, hi;
+  const Header* hdr;
+  int vec;
+  int unused;
+};
+
+__global__ void __launch_bounds__(kThreads) cast_allgather_kernel(const __grid_constant__ CastArgs a) {
+  __shared__ int s_run, s_live;
+  if (threadIdx.x == 0) {
+    int run = 1, live = 0;
+    if (a.gate == kGateNoOverflow) run = !__ldcg(&a.hdr->pending_flag);
+    if (a.gate == kGateRepair) {
+      run = __ldcg(&a.hdr->last_flag);
+      live = __ldcg(&a.hdr->live) & 1;
+    }
+    s_run = run;
+    s_live = live;
+  }
+  __syncthreads();
+  if (!s_run) return;
+  const float* __restrict__ src = a.src[s_live];
+  const Span sp8(a.lo, a.hi, a.vec);
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < sp8.nvec; j += stride) {
+    const int64_t i = sp8.vlo + (j << 3);
+    float P[8];
+    unpack(ld_stream(src + i), ld_stream(src + i + 4), P);
+    const uint4 w = pack_bf16x8(P);
+    for (int r = 0; r < a.nrep; ++r) st_stream(a.reps[r] + i, w);
+  }
+  for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
+    const int64_t i = sp8.scalar_index(a.lo, e);
+    const uint16_t w = to_bf16(src[i]);
+    for (int r = 0; r < a.nrep; ++r) a.reps[r][i] = w;
+  }
+}
+
+// ------------------------------------------------------------------ K2: ZeRO-3 layer gather
+
+struct GatherArgs {
+  const uint16_t* shards[kMaxNd];
+  uint16_t* out[kMaxNd];
+  int Nd, nout;
+  int64_t L, S;
+  int vec;  // S % 8 == 0 and every pointer 16-byte aligned
+  int unused;
+};
+
+// grid.y = source rank r; grid.x strides over the shard.  out[o][r*S + k] = shards[r][k].
+__global__ void __launch_bounds__(kThreads) gather_layer_kernel(const __grid_constant__ GatherArgs a) {
+  const int r = blockIdx.y;
+  const int64_t base = (int64_t)r * a.S;
+  int64_t len = a.L - base;  // real elements in shard r
+  if (len > a.S) len = a.S;
+  if (len <= 0) return;
+  const uint16_t* __restrict__ src = a.shards[r];
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  if (a.vec) {
+    const int64_t nvec = len >> 3;
+    for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < nvec; j += stride) {
+      const uint4 w = ld_stream(src + (j << 3));
+      for (int o = 0; o < a.nout; ++o) st_stream(a.out[o] + base + (j << 3), w);
+    }
+    const int64_t rest = len - (nvec << 3);
+    for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < rest; e += stride) {
+      const int64_t k = (nvec << 3) + e;
+      const uint16_t w = src[k];
+      for (int o = 0; o < a.nout; ++o) a.out[o][base + k] = w;
+    }
+  } else {
+    for (int64_t k = (int64_t)blockIdx.x * kThreads + threadIdx.x; k < len; k += stride) {
+      const uint16_t w = src[k];
+      for (int o = 0; o < a.nout; ++o) a.out[o][base + k] = w;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ workspace control
+
+enum : int { kWsInit = 0, kWsBegin = 1, kWsEnd = 2 };
+
+__global__ void ws_ctl_kernel(Header* h, int op, long long t0) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  if (op == kWsInit) {
+    h->done = 0u;
+    h->t = t0;
+    h->skipped = 0;
+    h->live = 0;
+    h->last_flag = 0;
+    h->last_sumsq = 0.0;
+  }
+  if (op == kWsInit || op == kWsBegin) {
+    h->pending_flag = 0;
+    h->pending_sumsq = 0.0;
+  }
+  if (op == kWsEnd) {
+    const int of = h->pending_flag;
+    h->last_flag = of;
+    h->last_sumsq = h->pending_sumsq;
+    if (!of)
+      h->t += 1;
+    else
+      h->skipped += 1;
+    h->pending_flag = 0;
+    h->pending_sumsq = 0.0;
+  }
+  __threadfence();
+}
+
+}  // namespace zb
