@@ -24,6 +24,7 @@
  *   - 16-bit values (gradients, bf16 weights) are passed as raw uint16_t bit patterns.
  *   - Pointers that are 16-byte aligned take the vectorised path; any other alignment is
  *     accepted and handled element by element (same results, slower).
+ *   - An empty window (lo == hi, N == 0, L == 0) is a valid no-op; its pointers may be NULL.
  *   - An overflow (inf/NaN in the reduced gradient) is not an error: the step is skipped and
  *     reported through the workspace (see zero_read_result).
  *   - Numerics: each update is the element-wise rule written out in zero_adam_shard, one

@@ -305,6 +305,7 @@ int zero_reduce_scatter(const uint16_t* const* grads, int dtype, int Nd, int64_t
   if ((rc = check_window(lo, hi))) return rc;
   if ((rc = check_hp(hp))) return rc;
   if (dtype != ZERO_BF16 && dtype != ZERO_FP16) return fail(ZERO_EINVAL, "dtype=%d", dtype);
+  if (lo == hi) return ZERO_OK;  // empty window: nothing to reduce or to report
   if (!grad_out || !ws) return fail(ZERO_EINVAL, "grad_out or workspace is NULL");
   zb::RsArgs a;
   std::memset(&a, 0, sizeof a);
@@ -328,6 +329,7 @@ int zero_adam_shard(float* master, float* exp_avg, float* exp_avg_sq, const floa
   int rc = check_window(lo, hi);
   if (rc) return rc;
   if ((rc = check_hp(hp))) return rc;
+  if (lo == hi) return ZERO_OK;
   if (!master || !exp_avg || !exp_avg_sq || !grad || !ws)
     return fail(ZERO_EINVAL, "master, exp_avg, exp_avg_sq, grad and workspace must be non-NULL");
   zb::AdamArgs a;
@@ -355,9 +357,10 @@ int zero_allgather(const float* master, uint16_t* const* replicas, int Nd, int64
   int rc = check_nd(Nd);
   if (rc) return rc;
   if ((rc = check_window(lo, hi))) return rc;
-  if (!master) return fail(ZERO_EINVAL, "master is NULL");
   if (gate != ZERO_GATE_ALWAYS && gate != ZERO_GATE_NO_OVERFLOW) return fail(ZERO_EINVAL, "gate=%d", gate);
   if (gate == ZERO_GATE_NO_OVERFLOW && !ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (lo == hi) return ZERO_OK;
+  if (!master) return fail(ZERO_EINVAL, "master is NULL");
   zb::CastArgs a;
   std::memset(&a, 0, sizeof a);
   bool al = aligned16(master);
