@@ -230,6 +230,46 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t *
  * by the caller.  Always returns ZERO_OK. */
 int zero_profile_events(void *start_event, void *stop_event);
 
+/* ------------------------------------------------------------------ no-allocation variant */
+
+/* Result of one zero_reduce_scatter_noalloc window (device memory owned by the caller). */
+typedef struct {
+    int32_t overflow;  /* 1 if any reduced element of the window is inf or NaN */
+    int32_t reserved;
+    double sumsq;      /* sum of squares of the window's reduced elements */
+} zero_rs_summary_t;
+
+#define ZERO_NOALLOC_MAX_CTAS 16384                                /* scratch slots */
+#define ZERO_NOALLOC_MAX_WINDOW ((int64_t)ZERO_NOALLOC_MAX_CTAS * 2048) /* 33,554,432 elements */
+
+/* The pages have no counterpart to this entry point: it exists for callers that cannot
+ * allocate device memory.  Some callers cannot hand the library a workspace: a plugin inside a
+ * host application that owns all device memory through its own fixed arena has no spare buffer
+ * to give, and code on a latency-critical path cannot call cudaMalloc, which may synchronize the
+ * whole device.  For them this call computes exactly what zero_reduce_scatter computes (the same
+ * grad_out, bit for bit) without a workspace and without allocating anything (no cudaMalloc,
+ * cudaFree or allocating library call).
+ *
+ * Its scratch -- one arrival counter and one partial (flag, sum of squares) per CTA -- is a fixed
+ * array inside the library: 256 B + 16 B x ZERO_NOALLOC_MAX_CTAS (about 256 KiB), held by every
+ * GPU that loads the library until the process exits.  The call uses one CTA per 2048 elements,
+ * so a window [lo, hi) may hold at most ZERO_NOALLOC_MAX_WINDOW elements; a larger window is
+ * rejected with ZERO_EINVAL and a message naming the limit (split it into buckets).
+ *
+ * grads, dtype, Nd, lo, hi, hp, grad_out: as for zero_reduce_scatter.  summary: device pointer the
+ * call writes the window's result to (accumulate = 0), or combines it into (accumulate != 0:
+ * overflow |= window's, sumsq += window's; the caller zeroes it before the first window).  The
+ * workspace bookkeeping of zero_step is not touched.
+ *
+ * The first call on each device looks up the scratch array's device address (with that device
+ * current) and keeps it; make that first call before any stream capture.  All calls share the one
+ * scratch array, which keeps the last call's contents; each call clears the counter before its
+ * kernel runs.  Calls that can overlap on the GPU (issued on different streams, or from different
+ * host threads without ordering) race on the scratch: issue them on one stream.  Async. */
+int zero_reduce_scatter_noalloc(const uint16_t *const *grads, int dtype, int Nd, int64_t lo,
+                                int64_t hi, const zero_hparams_t *hp, float *grad_out,
+                                zero_rs_summary_t *summary, int accumulate, void *stream);
+
 /* ------------------------------------------------------------------ accounting (host only) */
 
 /* Per-GPU model-state memory ([P1] §二 code: bytes_per_param for the 16-bit weights and again

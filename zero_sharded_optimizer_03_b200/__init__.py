@@ -17,7 +17,8 @@ __all__ = [
     "ZeroError", "zero_partition", "zero_workspace_bytes", "zero_workspace_init",
     "zero_read_result", "zero_begin_step", "zero_reduce_scatter", "zero_adam_shard",
     "zero_allgather", "zero_end_step", "zero3_gather_layer", "zero_step",
-    "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events", "hparams", "ZeroBuffers",
+    "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events",
+    "zero_reduce_scatter_noalloc", "ZERO_NOALLOC_MAX_WINDOW", "hparams", "ZeroBuffers",
     "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_GATE_ALWAYS",
     "ZERO_GATE_NO_OVERFLOW", "ZERO_MAX_ND",
 ]
@@ -59,6 +60,14 @@ class zero_state_t(ctypes.Structure):
                 ("workspace", _P)]
 
 
+class zero_rs_summary_t(ctypes.Structure):
+    _fields_ = [("overflow", _i32), ("reserved", _i32), ("sumsq", _dbl)]
+
+
+ZERO_NOALLOC_MAX_CTAS = 16384
+ZERO_NOALLOC_MAX_WINDOW = ZERO_NOALLOC_MAX_CTAS * 2048
+
+
 class zero_mem_t(ctypes.Structure):
     _fields_ = [("optimizer_states", _dbl), ("gradients", _dbl), ("parameters", _dbl),
                 ("total", _dbl)]
@@ -92,6 +101,9 @@ def _load() -> ctypes.CDLL:
                                   ctypes.POINTER(zero_mem_t)], ctypes.c_int),
         "zero_comm_volume": ([ctypes.c_int, _dbl, ctypes.c_int], _dbl),
         "zero_profile_events": ([_P, _P], ctypes.c_int),
+        "zero_reduce_scatter_noalloc": ([_P, ctypes.c_int, ctypes.c_int, _i64, _i64,
+                                         ctypes.POINTER(zero_hparams_t), _P, _P, ctypes.c_int,
+                                         _P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -172,6 +184,15 @@ def zero_adam_shard(master: int, exp_avg: int, exp_avg_sq: int, grad: int, lo: i
 def zero_allgather(master: int, replicas, Nd: int, lo: int, hi: int,
                    gate: int = ZERO_GATE_ALWAYS, ws: int | None = None, stream: int = 0) -> None:
     _check(lib.zero_allgather(master, _ptrs(replicas), Nd, lo, hi, gate, ws, stream))
+
+
+def zero_reduce_scatter_noalloc(grads, dtype: int, Nd: int, lo: int, hi: int,
+                                hp: zero_hparams_t, grad_out: int, summary: int,
+                                accumulate: bool = False, stream: int = 0) -> None:
+    """Workspace-free reduce-scatter (see include/zero.h): `summary` is a device pointer to a
+    zero_rs_summary_t (16 bytes) that receives the window's overflow flag and sum of squares."""
+    _check(lib.zero_reduce_scatter_noalloc(_ptrs(grads), dtype, Nd, lo, hi, ctypes.byref(hp),
+                                           grad_out, summary, 1 if accumulate else 0, stream))
 
 
 def zero_profile_events(start_event: int | None, stop_event: int | None) -> None:

@@ -570,3 +570,188 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
 }
 
 }  // extern "C"
+
+// ==================================================================== no-allocation variant
+//
+// zero_reduce_scatter_noalloc: the reduce-scatter of zero_reduce_scatter for callers that cannot
+// allocate device memory.  Its only scratch (the arrival counter and one partial per CTA) lives
+// in the file-scope array below instead of a caller-provided workspace.
+
+namespace {
+
+constexpr int kNoAllocTile = zb::kThreads * 8;  // elements per CTA: one 16-byte vector per thread
+constexpr size_t kNoAllocHeader = 256;          // arrival counter, padded to the array alignment
+constexpr size_t kNoAllocBytes = kNoAllocHeader + sizeof(zb::Partial) * ZERO_NOALLOC_MAX_CTAS;
+
+// Shared by every call on a device; held by every GPU that loads the library until exit.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+struct NoAllocRsArgs {
+  const uint16_t* grads[zb::kMaxNd];
+  float* out;
+  int64_t lo, hi;
+  float inv;
+  int Nd;
+  unsigned int* done;          // scratch: arrival counter (cleared before every launch)
+  zb::Partial* part;           // scratch: one slot per CTA
+  zero_rs_summary_t* summary;  // caller's output
+  int accumulate;
+  int vec;
+};
+
+template <int DT>
+__global__ void __launch_bounds__(zb::kThreads) reduce_scatter_noalloc_kernel(const __grid_constant__ NoAllocRsArgs a) {
+  double sq = 0.0;
+  int bad = 0;
+  float* __restrict__ out = a.out;
+  const zb::Span sp8(a.lo, a.hi, a.vec);
+  const int64_t stride = (int64_t)gridDim.x * zb::kThreads;
+  for (int64_t j = (int64_t)blockIdx.x * zb::kThreads + threadIdx.x; j < sp8.nvec; j += stride) {
+    const int64_t i = sp8.vlo + (j << 3);
+    float s[8];
+    zb::fan_in8<DT>(a.grads, a.Nd, i, s);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      s[k] = __fmul_rn(s[k], a.inv);
+      bad |= zb::nonfinite(s[k]);
+      sq = __dadd_rn(sq, __dmul_rn((double)s[k], (double)s[k]));
+    }
+    zb::st_stream(out + i, make_float4(s[0], s[1], s[2], s[3]));
+    zb::st_stream(out + i + 4, make_float4(s[4], s[5], s[6], s[7]));
+  }
+  for (int64_t e = (int64_t)blockIdx.x * zb::kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
+    const int64_t i = sp8.scalar_index(a.lo, e);
+    const float g = __fmul_rn(zb::fan_in1<DT>(a.grads, a.Nd, i), a.inv);
+    bad |= zb::nonfinite(g);
+    sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
+    out[i] = g;
+  }
+  // per-CTA partial into the scratch slot; the last CTA to arrive combines them in CTA order
+  __shared__ double r_sq[zb::kWarps];
+  __shared__ int r_bad[zb::kWarps];
+  __shared__ int am_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  sq = zb::warp_sum(sq);
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    r_sq[warp] = sq;
+    r_bad[warp] = bad;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    int f = 0;
+    for (int w = 0; w < zb::kWarps; ++w) {
+      s = __dadd_rn(s, r_sq[w]);
+      f |= r_bad[w];
+    }
+    a.part[blockIdx.x].sumsq = s;
+    a.part[blockIdx.x].flag = f;
+    __threadfence();
+    am_last = (atomicAdd(a.done, 1u) == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!am_last) return;
+  __threadfence();
+  double s = 0.0;
+  int f = 0;
+  for (int k = threadIdx.x; k < (int)gridDim.x; k += zb::kThreads) {
+    s = __dadd_rn(s, __ldcg(&a.part[k].sumsq));
+    f |= __ldcg(&a.part[k].flag);
+  }
+  s = zb::warp_sum(s);
+  f = __any_sync(0xffffffffu, f);
+  __syncthreads();
+  if (lane == 0) {
+    r_sq[warp] = s;
+    r_bad[warp] = f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    int fl = 0;
+    for (int w = 0; w < zb::kWarps; ++w) {
+      tot = __dadd_rn(tot, r_sq[w]);
+      fl |= r_bad[w];
+    }
+    if (a.accumulate) {
+      a.summary->overflow |= fl;
+      a.summary->sumsq = __dadd_rn(a.summary->sumsq, tot);
+    } else {
+      a.summary->overflow = fl;
+      a.summary->reserved = 0;
+      a.summary->sumsq = tot;
+    }
+  }
+}
+
+// Device address of the scratch array for the current device (looked up once per device).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(ZERO_EINVAL, "device ordinal %d unsupported", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return ZERO_OK;
+}
+
+}  // namespace
+
+extern "C" int zero_reduce_scatter_noalloc(const uint16_t* const* grads, int dtype, int Nd, int64_t lo, int64_t hi,
+                                           const zero_hparams_t* hp, float* grad_out, zero_rs_summary_t* summary,
+                                           int accumulate, void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if ((rc = check_window(lo, hi))) return rc;
+  if ((rc = check_hp(hp))) return rc;
+  if (dtype != ZERO_BF16 && dtype != ZERO_FP16) return fail(ZERO_EINVAL, "dtype=%d", dtype);
+  if (hi - lo > ZERO_NOALLOC_MAX_WINDOW)
+    return fail(ZERO_EINVAL,
+                "window of %lld elements exceeds the no-allocation limit of %lld elements "
+                "(%d scratch slots of %d elements); split it into smaller windows",
+                (long long)(hi - lo), (long long)ZERO_NOALLOC_MAX_WINDOW, ZERO_NOALLOC_MAX_CTAS, kNoAllocTile);
+  if (!summary) return fail(ZERO_EINVAL, "summary is NULL");
+  bool al = true;
+  if (hi > lo) {
+    if (!grad_out) return fail(ZERO_EINVAL, "grad_out is NULL");
+    al = aligned16(grad_out);
+    if ((rc = check_ptrs(grads, Nd, "grads", &al))) return rc;
+  }
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the arrival counter must start at zero; the partial slots are written before they are read
+  cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(unsigned int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counter)");
+  NoAllocRsArgs a;
+  std::memset(&a, 0, sizeof a);
+  if (hi > lo)
+    for (int r = 0; r < Nd; ++r) a.grads[r] = grads[r];
+  a.out = grad_out;
+  a.lo = lo;
+  a.hi = hi;
+  a.inv = make_consts(hp, Nd).inv;
+  a.Nd = Nd;
+  a.done = static_cast<unsigned int*>(scratch);
+  a.part = reinterpret_cast<zb::Partial*>(static_cast<unsigned char*>(scratch) + kNoAllocHeader);
+  a.summary = summary;
+  a.accumulate = accumulate != 0;
+  a.vec = al;
+  int64_t grid = (hi - lo + kNoAllocTile - 1) / kNoAllocTile;
+  if (grid < 1) grid = 1;  // an empty window still writes (or keeps) the summary
+  if (dtype == ZERO_FP16)
+    reduce_scatter_noalloc_kernel<1><<<(unsigned)grid, zb::kThreads, 0, s>>>(a);
+  else
+    reduce_scatter_noalloc_kernel<0><<<(unsigned)grid, zb::kThreads, 0, s>>>(a);
+  return check_launch("reduce_scatter_noalloc_kernel launch");
+}
