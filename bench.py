@@ -58,13 +58,27 @@ WORKLOADS = {
              "with m,v prefilled",
         stage=2, Nd=64, N=1 << 28, bucket=0, gdt="bf16", sigma=1e-3, kind="heavy", t0=999,
         hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
+    "zero3-llama7b": dict(
+        desc="ZeRO-3 Llama-7B-shaped: 32 layers of q,k,v,o 4096x4096 + gate,up,down 4096x11008 "
+             "(202,375,168 each), Nd=8; per layer gather from 8 bf16 shards and reduce-scatter "
+             "8 bf16 grad replicas ~N(0,1e-3) into the fp32 grad shard, then AdamW on the shards",
+        stage=3, Nd=8, N=32 * 202_375_168, layer=202_375_168, bucket=202_375_168, gdt="bf16",
+        sigma=1e-3, kind="normal",
+        hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
 }
 DEFAULT = "zero1-gpt2-small"
 
 
-def bytes_per_param(w) -> int:
+def bytes_per_param(w, two_pass=False) -> int:
+    Nd = w["Nd"]
+    if w["stage"] == 3:
+        # gather: 2 read + 2Nd written; RS: 2Nd read + 4 written; Adam + cast: 4 + 24 + 2
+        return (2 + 2 * Nd) + (2 * Nd + 4) + (4 + 24 + 2)
+    if two_pass:
+        # RS: 2Nd read + 4 written; Adam + cast + AG: 4 + 24 read/written + 2Nd written
+        return (2 * Nd + 4) + (4 + 24 + 2 * Nd)
     # fused step: Nd 2-byte gradient reads, fp32 master/m/v read + write, Nd 2-byte weight writes
-    return 2 * w["Nd"] + 24 + 2 * w["Nd"]
+    return 2 * Nd + 24 + 2 * Nd
 
 
 def peaks():
@@ -161,21 +175,49 @@ def cpu_baseline(w, target_s=10.0, steps=None):
         return grads, p, np.zeros(Np, np.float32), np.zeros(Np, np.float32), [
             np.zeros(n, np.uint16) for _ in range(Nd)]
 
+    def one_step(n, g, p, m, v, reps, t):
+        if w["stage"] == 3:  # the sample is one layer: gather, reduce-scatter, Adam + cast
+            sh16 = oracle.f32_to_bf16(p)
+            gathered = [np.zeros(n, np.uint16) for _ in range(Nd)]
+            return oracle.zero3_step(Nd, [n], odt, g, p, m, v, sh16, gathered, w["hp"], t)[0]
+        bucket = min(w.get("bucket", 0), n)
+        return oracle.zero12_step(Nd, n, bucket, odt, g, p, m, v, reps, w["hp"], t)[0]
+
     n0 = 1 << 18
     g, p, m, v, reps = make(n0)
     t = time.perf_counter()
-    oracle.zero12_step(Nd, n0, 0, odt, g, p, m, v, reps, w["hp"], 0)
+    one_step(n0, g, p, m, v, reps, 0)
     rate0 = n0 / (time.perf_counter() - t)
     n = int(min(w["N"], max(n0, rate0 * target_s)))
+    if w["stage"] == 3:
+        n -= n % Nd  # one unpadded layer
     g, p, m, v, reps = make(n)
     times = []
     tcount = 0
     for _ in range(steps or 1):
         t0 = time.perf_counter()
-        tcount, _, _ = oracle.zero12_step(Nd, n, w.get("bucket", 0), odt, g, p, m, v, reps,
-                                          w["hp"], tcount)
+        tcount = one_step(n, g, p, m, v, reps, tcount)
         times.append(time.perf_counter() - t0)
     return n, times
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity without dist).  Every
+    rank must call it with the same number of values, in the same order."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_rate(units_per_rank, world, ms_per_step):
+    """Units all ranks process per second when each rank processes units_per_rank per step and
+    the slowest rank takes ms_per_step (replicas: per-GPU work is fixed)."""
+    return world * units_per_rank / (ms_per_step / 1e3)
 
 
 # ----------------------------------------------------------------------------- main
@@ -192,6 +234,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--grad-sets-gb", type=float, default=24.0,
                     help="device memory budget for distinct per-step gradient sets")
+    ap.add_argument("--two-pass", action="store_true",
+                    help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather")
     ap.add_argument("--n-override", type=int, default=0,
                     help="run the workload at a different N (small cases for profiling)")
     args = ap.parse_args()
@@ -206,6 +250,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     config = {"workload": w["desc"], "N": w["N"], "Nd": w["Nd"], "stage": w["stage"],
               "bucket": w["bucket"], "grad_dtype": w["gdt"], "state_dtype": "f32",
+              "path": "two-pass" if args.two_pass else ("per-layer" if w["stage"] == 3 else "fused"),
               "weights_dtype": "bf16", "parallelism": "replicas (%d simulated ranks per GPU)"
               % w["Nd"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
               % (2 * w["Nd"] * w["N"] / 1e9)}
@@ -252,7 +297,13 @@ def main():
     kind = synth.HEAVY if w["kind"] == "heavy" else synth.NORMAL
     tail = float(__import__("numpy").float32(w["sigma"] * 1e3))
     hp = zero.hparams(**w["hp"])
-    buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt)
+    flags = zero.ZERO_TWO_PASS if args.two_pass else zero.ZERO_FUSED
+    if stage == 3:
+        assert w["layer"] % Nd == 0 and N % w["layer"] == 0, "unpadded layers expected"
+        buf = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, layer_len=w["layer"])
+    else:
+        buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt, flags=flags)
+    glen = buf.grads[0].numel()  # N (stages 1/2) or one layer (stage 3, reused per layer)
     synth.fill_device(buf.master[0].data_ptr(), synth.NORMAL, synth.F32, synth.SEED,
                       synth.MASTER_STREAM, N, 0.02, cuda_stream=sp)
     if w.get("t0"):
@@ -264,21 +315,28 @@ def main():
     buf.sync_params_from_master()
 
     # distinct gradient sets (set 0 lives in buf.grads)
-    set_bytes = 2 * Nd * N
+    set_bytes = 2 * Nd * glen
     nsets = int(max(1, min(args.warmup + args.steps, args.grad_sets_gb * 1e9 // set_bytes)))
-    gsets = [buf.grads] + [[torch.empty(N, dtype=buf.grads[0].dtype, device=dev)
+    if stage == 3:
+        nsets = 1
+    gsets = [buf.grads] + [[torch.empty(glen, dtype=buf.grads[0].dtype, device=dev)
                             for _ in range(Nd)] for _ in range(nsets - 1)]
     states = []
     for k, gs in enumerate(gsets):
         for r in range(Nd):
             synth.fill_device(gs[r].data_ptr(), kind, sdt, synth.SEED,
-                              synth.grad_stream(k + 1, r), N, w["sigma"], tail, cuda_stream=sp)
+                              synth.grad_stream(k + 1, r), glen, w["sigma"], tail, cuda_stream=sp)
         st = zero.zero_state_t.from_buffer_copy(buf.state)
         for r in range(Nd):
             st.grads[r] = gs[r].data_ptr()
         states.append(st)
     nb = 1 if w["bucket"] == 0 else -(-N // w["bucket"])
-    launches_per_step = nb + 1  # fused kernel per bucket + the overflow-repair check
+    if stage == 3:
+        launches_per_step = 3 * nb  # per layer: gather, reduce-scatter, Adam
+    elif args.two_pass:
+        launches_per_step = 2 * nb  # per bucket: reduce-scatter, Adam + all-gather
+    else:
+        launches_per_step = nb + 1  # fused kernel per bucket + the overflow-repair check
 
     def step(k, ev=None):
         if ev is not None:
@@ -316,24 +374,21 @@ def main():
     res = buf.result()
     assert res["overflow"] == 0 and res["skipped"] == 0, res
 
-    if dist:
-        t = torch.tensor([ms_total, kern_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, kern_ms = float(t[0]), float(t[1])
+    ms_total, kern_ms = max_over_ranks([ms_total, kern_ms], dist, dev)
     ms_step = ms_total / args.steps
-    value = world * N / (ms_step / 1e3)
-    bpp = bytes_per_param(w)
+    value = whole_job_rate(N, world, ms_step)
+    bpp = bytes_per_param(w, args.two_pass)
     achieved = bpp * N / (kern_ms / 1e3) / 1e9
     peak, peak_src = peaks()
     tr = traffic_record()
     traffic = None
-    if tr and tr.get("workload") == args.workload:
+    if tr and tr.get("workload") == args.workload and not args.two_pass and not args.n_override:
         traffic = tr["dram_bytes_per_launch"]
 
     # end to end through the public API: pinned host gradients -> device, step, result -> host
     e2e = None
     if not args.no_e2e:
-        host = [torch.empty(N, dtype=buf.grads[0].dtype, pin_memory=True) for _ in range(Nd)]
+        host = [torch.empty(glen, dtype=buf.grads[0].dtype, pin_memory=True) for _ in range(Nd)]
         for r in range(Nd):
             host[r].copy_(buf.grads[r])
         torch.cuda.synchronize()
@@ -351,13 +406,9 @@ def main():
             zero.zero_read_result(buf.ws.data_ptr(), sp)
         e_stop.record(s)
         torch.cuda.synchronize()
-        e_ms = e_start.elapsed_time(e_stop)
-        if dist:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t[0])
-        e2e = {"value": world * N / (e_ms / args.e2e_steps / 1e3), "unit": "params/s",
-               "h2d_bytes_per_step": 2 * Nd * N, "d2h_bytes_per_step": res_bytes,
+        e_ms = max_over_ranks([e_start.elapsed_time(e_stop)], dist, dev)[0]
+        e2e = {"value": whole_job_rate(N, world, e_ms / args.e2e_steps), "unit": "params/s",
+               "h2d_bytes_per_step": 2 * Nd * glen, "d2h_bytes_per_step": res_bytes,
                "steps": args.e2e_steps}
 
     cpu = None
@@ -374,7 +425,11 @@ def main():
                 "dtype": "f32", "data": "synthetic", "config": config,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                              "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                             "peak_source": peak_src, "kernel": "fused_step_kernel",
+                             "peak_source": peak_src,
+                             "kernel": ("zero3 step: gather_layer + reduce_scatter + adam kernels"
+                                        if stage == 3 else
+                                        "reduce_scatter + adam kernels (two-pass)"
+                                        if args.two_pass else "fused_step_kernel"),
                              "bytes_per_param": bpp, "kernel_ms": kern_ms,
                              "frac_of_8TBs": achieved / 8000.0},
                 "hbm_gbs_per_step": bpp * N / (ms_step / 1e3) / 1e9,
