@@ -89,18 +89,20 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def traffic_record():
-    """ncu DRAM bytes per launch of the fused kernel, valid only for the kernel source it was
-    captured from (profiles/traffic.json records that source's sha256)."""
+def traffic_record(kernel: str, workload: str):
+    """ncu DRAM bytes per launch of `kernel` on `workload` (profiles/traffic.json), or None when
+    no capture exists or a source file of the kernel has changed since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "zero_sharded_optimizer_03_b200", "csrc", "zero_kernels.cuh")
     if not os.path.exists(path):
         return None
-    rec = json.load(open(path))
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if rec.get("kernels_sha256") != sha:
-        return None
-    return rec
+    for rec in json.load(open(path)).get("records", []):
+        if rec.get("kernel") != kernel or rec.get("workload") != workload:
+            continue
+        for rel, sha in rec.get("sources", {}).items():
+            if hashlib.sha256(open(os.path.join(ROOT, rel), "rb").read()).hexdigest() != sha:
+                return None
+        return rec
+    return None
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -234,8 +236,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--grad-sets-gb", type=float, default=24.0,
                     help="device memory budget for distinct per-step gradient sets")
+    ap.add_argument("--no-tma", action="store_true",
+                    help="fused path: always the register-pipelined kernel")
+    ap.add_argument("--tma", action="store_true",
+                    help="fused path: always the TMA-pipelined kernel")
     ap.add_argument("--two-pass", action="store_true",
                     help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather")
+    ap.add_argument("--bucket-override", type=int, default=-1,
+                    help="stages 1/2: run with a different bucket size (0 = one bucket)")
     ap.add_argument("--n-override", type=int, default=0,
                     help="run the workload at a different N (small cases for profiling)")
     args = ap.parse_args()
@@ -244,13 +252,17 @@ def main():
     if args.n_override:
         w["N"] = args.n_override
         w["desc"] += " [N overridden to %d]" % args.n_override
+    if args.bucket_override >= 0 and w["stage"] != 3:
+        w["bucket"] = args.bucket_override
+        w["desc"] += " [bucket overridden to %d]" % args.bucket_override
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     config = {"workload": w["desc"], "N": w["N"], "Nd": w["Nd"], "stage": w["stage"],
               "bucket": w["bucket"], "grad_dtype": w["gdt"], "state_dtype": "f32",
-              "path": "two-pass" if args.two_pass else ("per-layer" if w["stage"] == 3 else "fused"),
+              "path": "two-pass" if args.two_pass else ("per-layer" if w["stage"] == 3 else
+                                                         "fused"),
               "weights_dtype": "bf16", "parallelism": "replicas (%d simulated ranks per GPU)"
               % w["Nd"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
               % (2 * w["Nd"] * w["N"] / 1e9)}
@@ -298,6 +310,20 @@ def main():
     tail = float(__import__("numpy").float32(w["sigma"] * 1e3))
     hp = zero.hparams(**w["hp"])
     flags = zero.ZERO_TWO_PASS if args.two_pass else zero.ZERO_FUSED
+    if args.no_tma:
+        flags |= zero.ZERO_NO_TMA
+    if args.tma:
+        flags |= zero.ZERO_FORCE_TMA
+    # which fused kernel zero_step picks (mirrors the library's rule)
+    tma_path = (not args.two_pass and w["stage"] != 3 and not args.no_tma and
+                (args.tma or (w["Nd"] >= 32 and (w["bucket"] or w["N"]) >= (1 << 26))))
+    if w["stage"] == 3:
+        line_kernel = "zero3 step: gather_layer + reduce_scatter + adam kernels"
+    elif args.two_pass:
+        line_kernel = "reduce_scatter + adam kernels (two-pass)"
+    else:
+        line_kernel = "fused_step_tma_kernel" if tma_path else "fused_step_kernel"
+    config["kernel"] = line_kernel
     if stage == 3:
         assert w["layer"] % Nd == 0 and N % w["layer"] == 0, "unpadded layers expected"
         buf = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, layer_len=w["layer"])
@@ -380,10 +406,10 @@ def main():
     bpp = bytes_per_param(w, args.two_pass)
     achieved = bpp * N / (kern_ms / 1e3) / 1e9
     peak, peak_src = peaks()
-    tr = traffic_record()
-    traffic = None
-    if tr and tr.get("workload") == args.workload and not args.two_pass and not args.n_override:
-        traffic = tr["dram_bytes_per_launch"]
+    tr = None
+    if not args.n_override and args.bucket_override < 0:
+        tr = traffic_record(line_kernel, args.workload)
+    traffic = tr["dram_bytes_per_launch"] if tr else None
 
     # end to end through the public API: pinned host gradients -> device, step, result -> host
     e2e = None
@@ -392,7 +418,7 @@ def main():
         for r in range(Nd):
             host[r].copy_(buf.grads[r])
         torch.cuda.synchronize()
-        res_bytes = 48  # the workspace header zero_read_result copies back
+        res_bytes = 56  # the workspace header zero_read_result copies back
         e_start = torch.cuda.Event(enable_timing=True)
         e_stop = torch.cuda.Event(enable_timing=True)
         if dist:
@@ -426,10 +452,7 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                              "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                              "peak_source": peak_src,
-                             "kernel": ("zero3 step: gather_layer + reduce_scatter + adam kernels"
-                                        if stage == 3 else
-                                        "reduce_scatter + adam kernels (two-pass)"
-                                        if args.two_pass else "fused_step_kernel"),
+                             "kernel": line_kernel,
                              "bytes_per_param": bpp, "kernel_ms": kern_ms,
                              "frac_of_8TBs": achieved / 8000.0},
                 "hbm_gbs_per_step": bpp * N / (ms_step / 1e3) / 1e9,

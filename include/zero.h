@@ -57,6 +57,8 @@ extern "C" {
 /* zero_step flags */
 #define ZERO_FUSED 0     /* stages 1/2: one fused pass (default); state copies ping-pong */
 #define ZERO_TWO_PASS 1  /* stages 1/2: reduce-scatter into grad_shard, then Adam + all-gather */
+#define ZERO_NO_TMA 2    /* ZERO_FUSED: always use the register-pipelined kernel */
+#define ZERO_FORCE_TMA 4 /* ZERO_FUSED: use the TMA-pipelined kernel whenever buffers are aligned */
 
 /* zero_allgather gates */
 #define ZERO_GATE_ALWAYS 0      /* always cast and write */
@@ -96,6 +98,9 @@ typedef struct {
     int32_t pending_overflow; /* overflow accumulated by the step in progress */
     int32_t reserved;
     double pending_sumsq;     /* sum of squares accumulated by the step in progress */
+    int32_t error;            /* nonzero if a kernel gave up a bounded internal wait (1 s); the
+                                 step was then skipped.  Sticky until zero_workspace_init. */
+    int32_t reserved2;
 } zero_step_result_t;
 
 /* Buffers of a whole step (zero_step).  All pointers are device pointers owned by the caller.
@@ -206,7 +211,11 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
 /* One optimizer step of ZeRO stage 1, 2 or 3 ([P1] §二 and §三; [P2] "ZeRO Stage 1/2/3").
  *   stage 1/2, ZERO_FUSED (default): reduce-scatter + unscale + overflow check + Adam + bf16
  *     cast + all-gather in one pass over each bucket [k*bucket, (k+1)*bucket) of [0, N)
- *     (bucket = 0: one bucket).  The pass reads state copy `live` and writes copy 1-live and
+ *     (bucket = 0: one bucket).  Two kernels implement the pass with identical results: a
+ *     register-pipelined one (16-byte vector loads and stores) and a TMA-pipelined one (bulk
+ *     copies through a shared-memory ring, bulk-store fan-out to the replicas).  The TMA one is
+ *     chosen for wide fan-in (Nd >= 32) over buckets of at least 2^26 elements when every buffer
+ *     is 16-byte aligned; ZERO_NO_TMA / ZERO_FORCE_TMA in flags override the choice.  The pass reads state copy `live` and writes copy 1-live and
  *     the Nd weight replicas; when the step ends without overflow the copies swap, otherwise
  *     the replicas are rewritten from the unchanged state.  Stages 1 and 2 compute the same
  *     values (they differ in what a real cluster keeps in memory, see zero_memory_estimate).
@@ -269,6 +278,15 @@ typedef struct {
 int zero_reduce_scatter_noalloc(const uint16_t *const *grads, int dtype, int Nd, int64_t lo,
                                 int64_t hi, const zero_hparams_t *hp, float *grad_out,
                                 zero_rs_summary_t *summary, int accumulate, void *stream);
+
+/* Test hook for the bounded waits inside the TMA-pipelined kernel (failure detection without a
+ * GPU fault).  The next TMA-pipelined launch made by zero_step on this thread issues no copies
+ * for load unit `unit` of its first CTA, so nothing ever completes that unit's barrier: the
+ * CTA's consumers give up after the 1 s bound, the launch drains what it issued, the workspace
+ * error word is set (zero_step_result_t.error) and the step is reported as overflowed, so the
+ * state and the weight replicas keep their values.  The device stays usable.  One-shot; -1
+ * clears.  Units of a CTA are numbered ceil(Nd/8) gradient chunks then one state unit per tile. */
+int zero_test_inject_stall(int64_t unit);
 
 /* ------------------------------------------------------------------ accounting (host only) */
 

@@ -117,6 +117,8 @@ CASES = [(0, 4), (1, 1), (1, 4), (7, 3), (8, 8), (9, 2), (15, 64), (17, 5), (100
 @pytest.mark.parametrize("N,Nd", CASES)
 @pytest.mark.parametrize("gdt", [zero.ZERO_BF16, zero.ZERO_FP16])
 @pytest.mark.parametrize("flags,bucket", [(zero.ZERO_FUSED, 0), (zero.ZERO_FUSED, 1001),
+                                          (zero.ZERO_FUSED | zero.ZERO_FORCE_TMA, 0),
+                                          (zero.ZERO_FUSED | zero.ZERO_FORCE_TMA, 5000),
                                           (zero.ZERO_TWO_PASS, 0), (zero.ZERO_TWO_PASS, 777)])
 def test_small_ragged_three_steps(N, Nd, gdt, flags, bucket):
     odt, sdt = DT[gdt]
@@ -182,6 +184,36 @@ def test_unaligned_views_take_the_scalar_path():
     assert_f32_close(states[4 + live].cpu().numpy(), vm, "unaligned exp_avg_sq")
     for r in range(Nd):
         assert_bf16_close(u16(reps[r]), oreps[r], "unaligned replica")
+
+
+@pytest.mark.parametrize("Nd,gdt", [(1, zero.ZERO_BF16), (8, zero.ZERO_BF16), (9, zero.ZERO_FP16),
+                                    (16, zero.ZERO_FP16), (64, zero.ZERO_BF16)])
+def test_tma_and_register_kernels_identical(Nd, gdt):
+    """The TMA-pipelined and register-pipelined fused kernels give the same bytes (whole tiles,
+    a ragged tail and an unaligned bucket start), and the same flag; sums of squares agree to
+    the reduction-order tolerance."""
+    N = 2048 * 301 + 1237
+    sdt = DT[gdt][1]
+    outs = []
+    for flags in (zero.ZERO_FUSED | zero.ZERO_FORCE_TMA, zero.ZERO_FUSED | zero.ZERO_NO_TMA):
+        buf = zero.ZeroBuffers(2, Nd, N, grad_dtype=gdt, flags=flags)
+        _init_state(buf, N, t0=3, m_kind=synth.ABS, v_kind=synth.SQUARE, m_sigma=1e-3,
+                    v_sigma=1e-6)
+        for k in (1, 2):
+            for r in range(Nd):
+                fill(buf.grads[r], synth.NORMAL, sdt, synth.grad_stream(k, r), sigma=1e-3)
+            buf.step(zero.hparams(**HP_C2), bucket=100_001)
+        res = buf.result()
+        live = buf.live()
+        outs.append((res, f32(buf.master[live]).tobytes(), f32(buf.exp_avg[live]).tobytes(),
+                     f32(buf.exp_avg_sq[live]).tobytes(),
+                     [u16(p).tobytes() for p in buf.params]))
+        del buf
+    (ra, *a), (rb, *b) = outs
+    assert a == b
+    assert (ra["step"], ra["overflow"], ra["error"]) == (rb["step"], rb["overflow"], 0) == (5, 0, 0)
+    assert abs(ra["grad_sumsq"] - rb["grad_sumsq"]) <= 1e-5 * rb["grad_sumsq"]
+    free()
 
 
 def test_stage1_and_stage2_identical():
@@ -271,6 +303,37 @@ def test_overflow_skips_then_recovers(flags, bad):
     t, _, ss = oracle.zero12_step(Nd, N, 0, oracle.BF16, hg, om, mm, vm, oreps, hp, t)
     res = _compare_full(buf, om, mm, vm, oreps, t, ss, "after skip")
     assert res["overflow"] == 0 and res["skipped"] == 1 and res["step"] == 12
+    del buf
+    free()
+
+
+def test_bounded_wait_gives_up_reports_error_and_device_stays_usable():
+    """A load that never lands (test hook: the producer of CTA 0 skips one unit) must not hang
+    the GPU: the consumers give up after 1 s, the step is skipped with the error word set, the
+    state and replicas keep their values, and the next step runs normally."""
+    Nd, N = 8, 2048 * 400
+    hp = dict(HP_C2)
+    buf = zero.ZeroBuffers(2, Nd, N, flags=zero.ZERO_FUSED | zero.ZERO_FORCE_TMA)
+    _init_state(buf, N)
+    for r in range(Nd):
+        fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(1, r), sigma=1e-3)
+    snap = [f32(buf.master[0]).tobytes()] + [u16(p).tobytes() for p in buf.params]
+    zero.zero_test_inject_stall(2)  # CTA 0, tile 1, its gradient chunk
+    buf.step(zero.hparams(**hp))
+    res = buf.result()
+    assert res["error"] != 0 and res["overflow"] == 1 and res["skipped"] == 1 and res["step"] == 0
+    assert res["live"] == 0
+    assert [f32(buf.master[0]).tobytes()] + [u16(p).tobytes() for p in buf.params] == snap
+    buf.step(zero.hparams(**hp))  # the hook was one-shot: this step commits
+    res = buf.result()
+    assert res["overflow"] == 0 and res["step"] == 1 and res["live"] == 1
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    grads = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(1, r), N,
+                             sigma=1e-3) for r in range(Nd)]
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    oracle.zero12_step(Nd, N, 0, oracle.BF16, grads, om, mm, vm, oreps, hp, 0)
+    assert_f32_close(f32(buf.master[1]), om, "after a timed-out step")
     del buf
     free()
 

@@ -18,8 +18,11 @@ __all__ = [
     "zero_read_result", "zero_begin_step", "zero_reduce_scatter", "zero_adam_shard",
     "zero_allgather", "zero_end_step", "zero3_gather_layer", "zero_step",
     "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events",
+    "zero_test_inject_stall",
     "zero_reduce_scatter_noalloc", "ZERO_NOALLOC_MAX_WINDOW", "hparams", "ZeroBuffers",
-    "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_GATE_ALWAYS",
+    "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_NO_TMA",
+    "ZERO_FORCE_TMA",
+    "ZERO_GATE_ALWAYS",
     "ZERO_GATE_NO_OVERFLOW", "ZERO_MAX_ND",
 ]
 
@@ -28,7 +31,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzero.so"
 ZERO_OK, ZERO_EINVAL, ZERO_ECUDA = 0, -1, -2
 ZERO_MAX_ND = 64
 ZERO_BF16, ZERO_FP16 = 0, 1
-ZERO_FUSED, ZERO_TWO_PASS = 0, 1
+ZERO_FUSED, ZERO_TWO_PASS, ZERO_NO_TMA, ZERO_FORCE_TMA = 0, 1, 2, 4
 ZERO_GATE_ALWAYS, ZERO_GATE_NO_OVERFLOW = 0, 1
 
 _i64, _i32, _dbl, _P = ctypes.c_int64, ctypes.c_int32, ctypes.c_double, ctypes.c_void_p
@@ -48,7 +51,7 @@ class zero_hparams_t(ctypes.Structure):
 class zero_step_result_t(ctypes.Structure):
     _fields_ = [("step", _i64), ("skipped", _i64), ("overflow", _i32), ("live", _i32),
                 ("grad_sumsq", _dbl), ("pending_overflow", _i32), ("reserved", _i32),
-                ("pending_sumsq", _dbl)]
+                ("pending_sumsq", _dbl), ("error", _i32), ("reserved2", _i32)]
 
 
 class zero_state_t(ctypes.Structure):
@@ -101,6 +104,7 @@ def _load() -> ctypes.CDLL:
                                   ctypes.POINTER(zero_mem_t)], ctypes.c_int),
         "zero_comm_volume": ([ctypes.c_int, _dbl, ctypes.c_int], _dbl),
         "zero_profile_events": ([_P, _P], ctypes.c_int),
+        "zero_test_inject_stall": ([_i64], ctypes.c_int),
         "zero_reduce_scatter_noalloc": ([_P, ctypes.c_int, ctypes.c_int, _i64, _i64,
                                          ctypes.POINTER(zero_hparams_t), _P, _P, ctypes.c_int,
                                          _P], ctypes.c_int),
@@ -162,7 +166,8 @@ def zero_workspace_init(ws: int, t: int = 0, stream: int = 0) -> None:
 def zero_read_result(ws: int, stream: int = 0) -> dict:
     out = zero_step_result_t()
     _check(lib.zero_read_result(ws, ctypes.byref(out), stream))
-    return {k: getattr(out, k) for k, _ in zero_step_result_t._fields_ if k != "reserved"}
+    return {k: getattr(out, k) for k, _ in zero_step_result_t._fields_
+            if not k.startswith("reserved")}
 
 
 def zero_begin_step(ws: int, stream: int = 0) -> None:
@@ -193,6 +198,10 @@ def zero_reduce_scatter_noalloc(grads, dtype: int, Nd: int, lo: int, hi: int,
     zero_rs_summary_t (16 bytes) that receives the window's overflow flag and sum of squares."""
     _check(lib.zero_reduce_scatter_noalloc(_ptrs(grads), dtype, Nd, lo, hi, ctypes.byref(hp),
                                            grad_out, summary, 1 if accumulate else 0, stream))
+
+
+def zero_test_inject_stall(unit: int) -> None:
+    _check(lib.zero_test_inject_stall(unit))
 
 
 def zero_profile_events(start_event: int | None, stop_event: int | None) -> None:
@@ -260,11 +269,11 @@ class ZeroBuffers:
             self.grads = [torch.zeros(N, dtype=gdt, device=device) for _ in range(Nd)]
             self.params = [torch.zeros(N, dtype=torch.bfloat16, device=device)
                            for _ in range(Nd)]
-            copies = 2 if flags == ZERO_FUSED else 1
+            copies = 1 if flags & ZERO_TWO_PASS else 2
             self.master = [torch.zeros(self.Np, **f32) for _ in range(copies)]
             self.exp_avg = [torch.zeros(self.Np, **f32) for _ in range(copies)]
             self.exp_avg_sq = [torch.zeros(self.Np, **f32) for _ in range(copies)]
-            self.grad_shard = (torch.zeros(self.Np, **f32) if flags == ZERO_TWO_PASS else None)
+            self.grad_shard = torch.zeros(self.Np, **f32) if flags & ZERO_TWO_PASS else None
             self.param_shard = None
         elif stage == 3:
             L = layer_len if layer_len > 0 else N
@@ -314,7 +323,8 @@ class ZeroBuffers:
         return zero_read_result(self.ws.data_ptr(), self.stream())
 
     def live(self) -> int:
-        return self.result()["live"] if self.flags == ZERO_FUSED and self.stage in (1, 2) else 0
+        fused = not (self.flags & ZERO_TWO_PASS)
+        return self.result()["live"] if fused and self.stage in (1, 2) else 0
 
     def sync_params_from_master(self) -> None:
         """Write bf16(master) into every weight replica (stage 1/2) or the bf16 shards

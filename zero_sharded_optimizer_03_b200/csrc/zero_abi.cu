@@ -13,6 +13,7 @@
 
 #include "zero.h"
 #include "zero_kernels.cuh"
+#include "zero_tma.cuh"
 
 namespace {
 
@@ -53,6 +54,7 @@ const void* kernel_ptr(int id) {
 struct DeviceInfo {
   int sms = 0;
   int per_sm[kNumKernels] = {};
+  bool tma_ready = false;  // dynamic shared memory attribute set for the TMA kernels
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -82,6 +84,31 @@ int grid_for(int kid, int64_t work, int* grid) {
   int64_t need = (work + zb::kThreads - 1) / zb::kThreads;
   if (need < 1) need = 1;
   *grid = (int)(need < cap ? need : cap);
+  return ZERO_OK;
+}
+
+// SM count of the current device, and the TMA kernels' shared-memory attribute set once.
+int tma_setup(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(ZERO_EINVAL, "device ordinal %d unsupported", dev);
+  DeviceInfo& d = g_dev[dev];
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (d.sms == 0) {
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+  if (!d.tma_ready) {
+    e = cudaFuncSetAttribute(zb::fused_step_tma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)zb::kTmaSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(zb::fused_step_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)zb::kTmaSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(TMA shared memory)");
+    d.tma_ready = true;
+  }
+  *sms = d.sms;
   return ZERO_OK;
 }
 
@@ -146,6 +173,7 @@ int check_ptrs(T* const* ptrs, int n, const char* what, bool* all_aligned) {
 
 // Optional CUDA events recorded around the data-moving kernels of the next zero_step call
 // on this thread (one-shot; see zero_profile_events).
+thread_local int64_t g_test_stall = -1;  // zero_test_inject_stall (one-shot)
 thread_local cudaEvent_t g_prof_start = nullptr;
 thread_local cudaEvent_t g_prof_stop = nullptr;
 
@@ -169,6 +197,26 @@ int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s) {
   else
     zb::fused_step_kernel<0><<<grid, zb::kThreads, 0, s>>>(a);
   return check_launch("fused_step_kernel launch");
+}
+
+// TMA-pipelined fused step over [a.lo, a.hi): whole tiles through the bulk-copy pipeline, the
+// rest by the same kernel's consumers.  Every pointer must be 16-byte aligned.
+int launch_fused_tma(int dtype, zb::TmaArgs& a, cudaStream_t s) {
+  int sms = 0;
+  int rc = tma_setup(&sms);
+  if (rc) return rc;
+  a.tiles_lo = (a.lo + 7) & ~int64_t(7);
+  if (a.tiles_lo > a.hi) a.tiles_lo = a.hi;
+  a.ntiles = (a.hi - a.tiles_lo) / zb::kTile;
+  int64_t grid = a.ntiles < sms ? a.ntiles : sms;
+  if (grid < 1) grid = 1;
+  a.stall_unit = g_test_stall;
+  g_test_stall = -1;
+  if (dtype == ZERO_FP16)
+    zb::fused_step_tma_kernel<1><<<(unsigned)grid, zb::kTmaThreads, zb::kTmaSmemBytes, s>>>(a);
+  else
+    zb::fused_step_tma_kernel<0><<<(unsigned)grid, zb::kTmaThreads, zb::kTmaSmemBytes, s>>>(a);
+  return check_launch("fused_step_tma_kernel launch");
 }
 
 int launch_rs(int dtype, const zb::RsArgs& a, cudaStream_t s) {
@@ -279,12 +327,20 @@ int zero_read_result(const void* ws, zero_step_result_t* out, void* stream) {
   out->pending_overflow = h.pending_flag;
   out->reserved = 0;
   out->pending_sumsq = h.pending_sumsq;
+  out->error = h.error;
+  out->reserved2 = 0;
   return ZERO_OK;
 }
 
 int zero_profile_events(void* start_event, void* stop_event) {
   g_prof_start = (cudaEvent_t)start_event;
   g_prof_stop = (cudaEvent_t)stop_event;
+  return ZERO_OK;
+}
+
+int zero_test_inject_stall(int64_t unit) {
+  if (unit < -1) return fail(ZERO_EINVAL, "unit=%lld < -1", (long long)unit);
+  g_test_stall = unit;
   return ZERO_OK;
 }
 
@@ -546,12 +602,41 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   a.part = partials(ws);
   a.Nd = Nd;
   a.vec = al;
+  // The TMA pipeline wins only where many loads must be in flight per element: a wide fan-in
+  // over a long window (measured on B200: +1.2% at Nd = 64 over 2^28 elements; -1..-3% at
+  // Nd = 8..16, and a fixed cost per launch that hurts short bucketed windows).
+  const bool tma_auto = Nd >= 32 && B >= (int64_t(1) << 26);
+  const bool tma = al && !(st->flags & ZERO_NO_TMA) && ((st->flags & ZERO_FORCE_TMA) || tma_auto);
+  zb::TmaArgs ta;
+  if (tma) {
+    std::memset(&ta, 0, sizeof ta);
+    for (int r = 0; r < Nd; ++r) {
+      ta.grads[r] = a.grads[r];
+      ta.reps[r] = a.reps[r];
+    }
+    for (int i = 0; i < 2; ++i) {
+      ta.p[i] = a.p[i];
+      ta.m[i] = a.m[i];
+      ta.v[i] = a.v[i];
+    }
+    ta.c = c;
+    ta.hdr = a.hdr;
+    ta.part = a.part;
+    ta.Nd = Nd;
+  }
   prof_mark(true, s);
   for (int64_t k = 0; k < nb; ++k) {
     a.lo = k * B < N ? k * B : N;
     a.hi = (k + 1) * B < N ? (k + 1) * B : N;
     a.mode = (k == 0 ? zb::kAccSet : zb::kAccAdd) | (k == nb - 1 ? (zb::kFinalize | zb::kFlip) : 0);
-    if ((rc = launch_fused(st->grad_dtype, a, s))) return rc;
+    if (tma) {
+      ta.lo = a.lo;
+      ta.hi = a.hi;
+      ta.mode = a.mode;
+      if ((rc = launch_fused_tma(st->grad_dtype, ta, s))) return rc;
+    } else if ((rc = launch_fused(st->grad_dtype, a, s))) {
+      return rc;
+    }
   }
   prof_mark(false, s);
   // overflow repair: rewrite the replicas from the unchanged state (runs only after a skip)

@@ -41,6 +41,8 @@ struct Header {
   int live;               // state copy holding the current state (fused path)
   int last_flag;          // overflow of the last finished step
   double last_sumsq;      // sum of squares of the last finished step
+  int error;              // nonzero once a kernel gave up a bounded wait (sticky until init)
+  int unused;
 };
 static_assert(sizeof(Header) <= 256, "header must fit its slot");
 
@@ -234,10 +236,11 @@ __device__ __forceinline__ double warp_sum(double x) {
 // Launch epilogue: per-CTA totals into the partials, and the last CTA to arrive reduces them
 // in CTA order and applies `mode` to the header.  No CTA waits for another (the last one to
 // arrive does the work), so there is no spin and no co-residency assumption.
+template <int NW = kWarps>
 __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Partial* part, int mode) {
   if (mode == 0) return;
-  __shared__ double r_sq[kWarps];
-  __shared__ int r_bad[kWarps];
+  __shared__ double r_sq[NW];
+  __shared__ int r_bad[NW];
   __shared__ int am_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   sq = warp_sum(sq);
@@ -250,7 +253,7 @@ __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Pa
   if (threadIdx.x == 0) {
     double s = 0.0;
     int f = 0;
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       s = __dadd_rn(s, r_sq[w]);
       f |= r_bad[w];
     }
@@ -265,7 +268,7 @@ __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Pa
   __threadfence();
   double s = 0.0;
   int f = 0;
-  for (int k = threadIdx.x; k < (int)gridDim.x; k += kThreads) {
+  for (int k = threadIdx.x; k < (int)gridDim.x; k += NW * 32) {
     s = __dadd_rn(s, __ldcg(&part[k].sumsq));
     f |= __ldcg(&part[k].flag);
   }
@@ -280,7 +283,7 @@ __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Pa
   if (threadIdx.x == 0) {
     double tot = 0.0;
     int fl = 0;
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       tot = __dadd_rn(tot, r_sq[w]);
       fl |= r_bad[w];
     }
@@ -607,6 +610,7 @@ __global__ void ws_ctl_kernel(Header* h, int op, long long t0) {
     h->live = 0;
     h->last_flag = 0;
     h->last_sumsq = 0.0;
+    h->error = 0;
   }
   if (op == kWsInit || op == kWsBegin) {
     h->pending_flag = 0;
