@@ -89,6 +89,15 @@ def lib() -> ctypes.CDLL:
         L.oracle_zero3_step.restype = i32
         L.oracle_update_elements.argtypes = [i32, i64, i32, P, P, P, P, P, P, P, i64, i32]
         L.oracle_update_elements.restype = None
+        L.oracle_scaler_update.argtypes = [P, P, i32, dbl, dbl, i64]
+        L.oracle_scaler_update.restype = None
+        L.oracle_clip_coef.argtypes = [dbl, dbl]
+        L.oracle_clip_coef.restype = ctypes.c_float
+        L.oracle_zero12_step_ex.argtypes = [i32, i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P]
+        L.oracle_zero12_step_ex.restype = i32
+        L.oracle_update_elements_ex.argtypes = [i32, i64, i32, P, P, P, P, P, P, i64, i32,
+                                                ctypes.c_float]
+        L.oracle_update_elements_ex.restype = None
         L.oracle_memory_estimate.argtypes = [dbl, i32, i32, i32, P]
         L.oracle_memory_estimate.restype = None
         L.oracle_comm_volume.argtypes = [i32, dbl, i32]
@@ -255,6 +264,52 @@ def update_elements(Nd, dtype, grads_en, p, m, v, hp, t_new, skip, want_grad=Fal
                                  None if gout is None else _ptr(gout), _ptr(_hp(hp)), t_new,
                                  1 if skip else 0)
     return out16, gout
+
+
+def scaler_update(scale: float, good: int, overflow: bool, growth: float = 2.0,
+                  backoff: float = 0.5, interval: int = 2000):
+    """One dynamic loss-scale update.  Returns (scale, good)."""
+    sc = ctypes.c_double(scale)
+    gd = ctypes.c_int64(good)
+    lib().oracle_scaler_update(ctypes.byref(sc), ctypes.byref(gd), 1 if overflow else 0, growth,
+                               backoff, interval)
+    return sc.value, gd.value
+
+
+def clip_coef(sumsq: float, max_norm: float) -> float:
+    return float(lib().oracle_clip_coef(sumsq, max_norm))
+
+
+def _hpx(hp: dict) -> np.ndarray:
+    return np.concatenate([_hp(hp), np.array(
+        [hp.get("max_grad_norm", 0.0), hp.get("scale_growth", 2.0), hp.get("scale_backoff", 0.5),
+         float(hp.get("scale_interval", 2000)), 1.0 if hp.get("dynamic_scale", False) else 0.0],
+        dtype=np.float64)])
+
+
+def zero12_step_ex(Nd, N, bucket, dtype, grads, master, m, v, replicas, hp, t, scale=None, good=0):
+    """ZeRO-1/2 step with clipping (hp['max_grad_norm']) and, if hp['dynamic_scale'], the
+    dynamic loss scale `scale` / `good`.  Returns (t, overflow, sumsq, scale, good)."""
+    tt = ctypes.c_int64(t)
+    ovf = ctypes.c_int(0)
+    ss = ctypes.c_double(0.0)
+    sc = ctypes.c_double(hp.get("loss_scale", 1.0) if scale is None else scale)
+    gd = ctypes.c_int64(good)
+    rc = lib().oracle_zero12_step_ex(Nd, N, bucket, dtype, _ptr_array(grads), _ptr(master), _ptr(m),
+                                     _ptr(v), _ptr_array(replicas), _ptr(_hpx(hp)),
+                                     ctypes.byref(tt), ctypes.byref(sc), ctypes.byref(gd),
+                                     ctypes.byref(ovf), ctypes.byref(ss))
+    if rc != 0:
+        raise ValueError("oracle_zero12_step_ex failed")
+    return tt.value, ovf.value, ss.value, sc.value, gd.value
+
+
+def update_elements_ex(Nd, dtype, grads_en, p, m, v, hp, t_new, skip, coef):
+    g = np.ascontiguousarray(grads_en, dtype=np.uint16)
+    out16 = np.empty(p.size, dtype=np.uint16)
+    lib().oracle_update_elements_ex(Nd, p.size, dtype, _ptr(g), _ptr(p), _ptr(m), _ptr(v),
+                                    _ptr(out16), _ptr(_hp(hp)), t_new, 1 if skip else 0, coef)
+    return out16
 
 
 STAGES = ("DP", "ZeRO-1", "ZeRO-2", "ZeRO-3")

@@ -463,3 +463,100 @@ void oracle_f32_array_to_bf16(const float *src, uint16_t *dst, int64_t n)
 {
     for (int64_t i = 0; i < n; i++) dst[i] = oracle_f32_to_bf16(src[i]);
 }
+
+/* ---------------------------------------------------------------- loss scaler and clipping */
+
+/* Dynamic loss scaling (the pages only name mixed precision, [P3] "vs 混合精度"; reading: the
+ * standard backoff / growth rule).  After a step that overflowed, the scale is multiplied by
+ * `backoff` and the count of clean steps restarts; after `interval` clean steps in a row it is
+ * multiplied by `growth`, unless that would take it past the largest finite fp32 value (the
+ * scale multiplies fp32 losses, so it must stay finite there). */
+void oracle_scaler_update(double *scale, int64_t *good, int overflow, double growth, double backoff,
+                          int64_t interval)
+{
+    const double fp32_max = 3.4028234663852886e38;
+    if (overflow) {
+        *scale = *scale * backoff;
+        *good = 0;
+        return;
+    }
+    *good = *good + 1;
+    if (*good >= interval) {
+        double grown = *scale * growth;
+        if (grown <= fp32_max) *scale = grown;
+        *good = 0;
+    }
+}
+
+/* Global-norm clipping factor (reading: the usual rule, g <- g * min(1, max_norm/(||g|| + 1e-6)),
+ * with ||g|| the 2-norm of the whole reduced, unscaled gradient).  Evaluated in double, rounded
+ * once to fp32; 1 when max_norm <= 0 (no clipping). */
+float oracle_clip_coef(double sumsq, double max_norm)
+{
+    if (!(max_norm > 0.0)) return 1.0f;
+    double coef = max_norm / (sqrt(sumsq) + 1e-6);
+    if (coef > 1.0) coef = 1.0;
+    return (float)coef;
+}
+
+/* ZeRO-1/2 step with the two extensions.  hpx = {lr, beta1, beta2, eps, weight_decay,
+ * loss_scale, grad_average, max_grad_norm, growth, backoff, interval, dynamic}.  With dynamic
+ * != 0 the gradients carry the scale *scale (updated on return, with *good) instead of
+ * hpx[5].  Order: reduce-scatter (mean, unscaled), overflow check, clipping of the reduced
+ * gradient, Adam per shard, all-gather, scaler update. */
+int oracle_zero12_step_ex(int Nd, int64_t N, int64_t bucket, int dtype, const uint16_t *const *grads,
+                          float *master, float *m, float *v, uint16_t *const *replicas,
+                          const double hpx[12], int64_t *t, double *scale, int64_t *good,
+                          int *overflow, double *sumsq)
+{
+    int64_t part[3];
+    if (oracle_partition(N, Nd, part) != 0 || bucket < 0) return -1;
+    int64_t S = part[0], Np = part[1];
+    double hp[7];
+    for (int k = 0; k < 7; k++) hp[k] = hpx[k];
+    int dynamic = hpx[11] != 0.0;
+    if (dynamic) hp[5] = *scale;
+    float *g = (float *)malloc((size_t)(Np > 0 ? Np : 1) * sizeof(float));
+    if (!g) return -1;
+    oracle_scalars_t c;
+    oracle_scalars(hp, Nd, 1, &c);
+    *overflow = 0;
+    *sumsq = 0.0;
+    int64_t w = bucket > 0 ? bucket : (Np > 0 ? Np : 1);
+    for (int64_t lo = 0; lo < Np; lo += w) {
+        int64_t hi = lo + w < Np ? lo + w : Np;
+        oracle_reduce_scatter_window(Nd, N, dtype, grads, c.inv, lo, hi, g, overflow, sumsq);
+    }
+    if (!*overflow) {
+        float coef = oracle_clip_coef(*sumsq, hpx[7]);
+        for (int64_t i = 0; i < N; i++) g[i] = g[i] * coef;
+        *t = *t + 1;
+        oracle_scalars(hp, Nd, *t, &c);
+        for (int r = 0; r < Nd; r++) {
+            int64_t off = (int64_t)r * S;
+            oracle_adam(master + off, m + off, v + off, g + off, shard_len(N, S, r), &c);
+        }
+        oracle_allgather(Nd, N, master, replicas);
+    }
+    if (dynamic) oracle_scaler_update(scale, good, *overflow, hpx[8], hpx[9], (int64_t)hpx[10]);
+    free(g);
+    return 0;
+}
+
+/* Sampled-element form of the extended step: element e's gradients, state and result as in
+ * oracle_update_elements; the caller supplies the overflow decision, the clipping factor and
+ * the loss scale of the full vector. */
+void oracle_update_elements_ex(int Nd, int64_t n, int dtype, const uint16_t *grads, float *p, float *m,
+                               float *v, uint16_t *out16, const double hp[7], int64_t t_new,
+                               int skip, float coef)
+{
+    oracle_scalars_t c;
+    oracle_scalars(hp, Nd, t_new, &c);
+    for (int64_t e = 0; e < n; e++) {
+        float s = 0.0f;
+        for (int q = 0; q < Nd; q++) s = s + grad_value(grads, e * Nd + q, dtype);
+        float g = (s * c.inv) * coef;
+        if (!skip) oracle_adam(p + e, m + e, v + e, &g, 1, &c);
+        out16[e] = oracle_f32_to_bf16(p[e]);
+    }
+}
