@@ -418,7 +418,7 @@ def main():
         for r in range(Nd):
             host[r].copy_(buf.grads[r])
         torch.cuda.synchronize()
-        res_bytes = 56  # the workspace header zero_read_result copies back
+        res_bytes = 104  # the workspace header zero_read_result copies back
         e_start = torch.cuda.Event(enable_timing=True)
         e_stop = torch.cuda.Event(enable_timing=True)
         if dist:

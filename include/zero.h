@@ -83,9 +83,14 @@ typedef struct {
     double beta1, beta2;
     double eps;
     double weight_decay;  /* decoupled (AdamW); 0 gives Adam */
-    double loss_scale;    /* static fp16 loss scale the gradients carry; 1 if none */
+    double loss_scale;    /* static fp16 loss scale the gradients carry; 1 if none (ignored
+                             while the workspace's dynamic loss scaler is on) */
     int32_t grad_average; /* nonzero: g = sum/(Nd*loss_scale) (data-parallel mean); 0: sum/loss_scale */
     int32_t reserved;
+    double max_grad_norm; /* > 0: clip the reduced gradient to this global 2-norm before the
+                             update, g *= min(1, max_grad_norm/(||g|| + 1e-6)); 0: no clipping.
+                             Needs the norm before the update: ZERO_TWO_PASS, stage 3, or the
+                             building blocks (the fused one-pass step refuses it) */
 } zero_hparams_t;
 
 /* Host copy of the step bookkeeping kept in the workspace. */
@@ -101,6 +106,11 @@ typedef struct {
     int32_t error;            /* nonzero if a kernel gave up a bounded internal wait (1 s); the
                                  step was then skipped.  Sticky until zero_workspace_init. */
     int32_t reserved2;
+    double loss_scale;        /* dynamic loss scaler: the scale the next step's gradients must
+                                 carry (0 when the scaler is off) */
+    int64_t good_steps;       /* dynamic loss scaler: clean steps since the scale last changed */
+    int32_t dynamic_scale;    /* 1 when the dynamic loss scaler is on */
+    int32_t reserved3;
 } zero_step_result_t;
 
 /* Buffers of a whole step (zero_step).  All pointers are device pointers owned by the caller.
@@ -150,6 +160,16 @@ size_t zero_workspace_bytes(void);
 
 /* Sets the workspace to "t completed updates, nothing pending, state copy 0 live".  Async. */
 int zero_workspace_init(void *ws, int64_t t, void *stream);
+
+/* Turns on dynamic loss scaling for the optimizer that owns `ws` (mixed precision: the pages
+ * only name AMP, [P3] comparisons; this is the usual backoff/growth rule).  From then on the
+ * gradients of every step are taken to carry the workspace's current scale (hp->loss_scale is
+ * ignored) and the end of each step updates it: after an overflow (the step is skipped) scale *=
+ * backoff_factor; after growth_interval clean steps in a row scale *= growth_factor, unless that
+ * would leave the finite fp32 range.  Read the scale for the next backward pass from
+ * zero_read_result.  zero_workspace_init turns the scaler off.  Async. */
+int zero_loss_scaler_init(void *ws, double init_scale, double growth_factor, double backoff_factor,
+                          int64_t growth_interval, void *stream);
 
 /* Copies the workspace bookkeeping to *out.  Synchronizes `stream` (waits for queued steps). */
 int zero_read_result(const void *ws, zero_step_result_t *out, void *stream);
@@ -268,7 +288,8 @@ typedef struct {
  * grads, dtype, Nd, lo, hi, hp, grad_out: as for zero_reduce_scatter.  summary: device pointer the
  * call writes the window's result to (accumulate = 0), or combines it into (accumulate != 0:
  * overflow |= window's, sumsq += window's; the caller zeroes it before the first window).  The
- * workspace bookkeeping of zero_step is not touched.
+ * workspace bookkeeping of zero_step is not touched, so a dynamic loss scale kept there does not
+ * apply: the unscale factor comes from hp->loss_scale.
  *
  * The first call on each device looks up the scratch array's device address (with that device
  * current) and keeps it; make that first call before any stream capture.  All calls share the one

@@ -99,9 +99,29 @@ def test_entry_points_validate_before_touching_the_device(zero):
         lambda: zero.zero3_gather_layer([16] * 2, 2, -1, [16]),
         lambda: zero.zero_workspace_init(None, 0),
         lambda: zero.zero_workspace_init(16, -3),
+        lambda: zero.zero_step(1, 4, 10, 0, st, zero.hparams(1e-3, max_grad_norm=-1.0)),
+        lambda: zero.zero_loss_scaler_init(None, 1024.0),
+        lambda: zero.zero_loss_scaler_init(16, 0.0),
+        lambda: zero.zero_loss_scaler_init(16, 1024.0, growth_factor=0.5),
+        lambda: zero.zero_loss_scaler_init(16, 1024.0, backoff_factor=1.5),
+        lambda: zero.zero_loss_scaler_init(16, 1024.0, growth_interval=0),
+        lambda: zero.zero_test_inject_stall(-2),
     ]
     for k, call in enumerate(cases):
         with pytest.raises(zero.ZeroError) as e:
             call()
         assert e.value.code == zero.ZERO_EINVAL, k
         assert zero.lib.zero_last_error().decode() != ""
+
+
+def test_fused_step_refuses_clipping(zero):
+    st = zero.zero_state_t()
+    st.grad_dtype = zero.ZERO_BF16
+    st.flags = zero.ZERO_FUSED
+    for r in range(4):  # fake, never dereferenced: the call is refused before any device work
+        st.grads[r] = 4096
+        st.params[r] = 4096
+    st.workspace = 4096
+    with pytest.raises(zero.ZeroError) as e:
+        zero.zero_step(1, 4, 1000, 0, st, zero.hparams(1e-3, max_grad_norm=1.0))
+    assert e.value.code == zero.ZERO_EINVAL and "ZERO_TWO_PASS" in str(e.value)

@@ -338,6 +338,103 @@ def test_bounded_wait_gives_up_reports_error_and_device_stays_usable():
     free()
 
 
+# ----------------------------------------------------------------------------- scaler, clipping
+
+@pytest.mark.parametrize("flags", [zero.ZERO_FUSED, zero.ZERO_FUSED | zero.ZERO_FORCE_TMA,
+                                   zero.ZERO_TWO_PASS])
+def test_dynamic_loss_scaler_matches_oracle(flags):
+    """fp16 gradients carrying the workspace's loss scale; an overflow on step 3 halves the
+    scale and skips; two clean steps double it.  Every element and the scale sequence."""
+    Nd, N = 4, 2048 * 60 + 5
+    hp = dict(lr=1e-3, weight_decay=0.01, dynamic_scale=True, scale_interval=2,
+              scale_growth=2.0, scale_backoff=0.5)
+    buf = zero.ZeroBuffers(2, Nd, N, grad_dtype=zero.ZERO_FP16, flags=flags)
+    _init_state(buf, N)
+    zero.zero_loss_scaler_init(buf.ws.data_ptr(), 1024.0, 2.0, 0.5, 2, stream())
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    oreps = [oracle.f32_to_bf16(om[:N]) for _ in range(Nd)]
+    t, scale, good = 0, 1024.0, 0
+    seen = []
+    for k in range(1, 7):
+        res = buf.result()
+        assert res["dynamic_scale"] == 1 and res["loss_scale"] == scale
+        sigma = float(np.float32(1e-4 * scale))
+        hg = [synth.fill_host(synth.NORMAL, synth.FP16, SEED, synth.grad_stream(k, r), N,
+                              sigma=sigma) for r in range(Nd)]
+        for r in range(Nd):
+            fill(buf.grads[r], synth.NORMAL, synth.FP16, synth.grad_stream(k, r), sigma=sigma)
+        if k == 3:
+            put_bits(buf.grads[2], 777, 0x7C00)
+            hg[2][777] = 0x7C00
+        buf.step(zero.hparams(lr=1e-3, weight_decay=0.01))
+        t, ovf, ss, scale, good = oracle.zero12_step_ex(Nd, N, 0, oracle.FP16, hg, om, mm, vm,
+                                                        oreps, hp, t, scale, good)
+        res = buf.result()
+        assert res["overflow"] == ovf == (1 if k == 3 else 0)
+        assert (res["loss_scale"], res["good_steps"]) == (scale, good)
+        seen.append(scale)
+    assert seen == [1024.0, 2048.0, 1024.0, 1024.0, 2048.0, 2048.0]
+    _compare_full(buf, om, mm, vm, oreps, t, ss, "dynamic scale")
+    del buf
+    free()
+
+
+@pytest.mark.parametrize("Nd,N,bucket", [(8, 300_007, 0), (3, 100_003, 20_001)])
+def test_clipping_two_pass_matches_oracle(Nd, N, bucket):
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=1.0, max_grad_norm=0.05)
+    buf = zero.ZeroBuffers(2, Nd, N, flags=zero.ZERO_TWO_PASS)
+    _init_state(buf, N)
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t = 0
+    for k in (1, 2, 3):
+        hg = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(k, r), N,
+                              sigma=1e-3) for r in range(Nd)]
+        for r in range(Nd):
+            fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(k, r), sigma=1e-3)
+        buf.step(zero.hparams(lr=1e-3, weight_decay=0.01, max_grad_norm=0.05), bucket=bucket)
+        t, ovf, ss, _, _ = oracle.zero12_step_ex(Nd, N, bucket, oracle.BF16, hg, om, mm, vm, oreps,
+                                                 hp, t)
+        assert np.sqrt(ss) > 0.05  # clipping is active
+    _compare_full(buf, om, mm, vm, oreps, t, ss, "clipped two-pass")
+    del buf
+    free()
+
+
+def test_clipping_zero3_matches_flat_oracle():
+    """ZeRO-3 computes what unsharded data parallelism computes, so the clipped ZeRO-3 step on
+    unpadded layers equals the clipped flat step on the concatenated gradients."""
+    Nd, L, nl = 4, 4096, 3
+    N = L * nl
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=1.0, max_grad_norm=0.01)
+    buf = zero.ZeroBuffers(3, Nd, N, layer_len=L, per_layer_buffers=True)
+    om = synth.fill_host(synth.NORMAL, synth.F32, SEED, synth.MASTER_STREAM, N, sigma=0.02)
+    buf.master[0].copy_(torch.from_numpy(om))
+    buf.init_workspace(0)
+    buf.sync_params_from_master()
+    mm = np.zeros(N, np.float32)
+    vm = np.zeros(N, np.float32)
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t = 0
+    for k in (1, 2):
+        flat = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(k, r), N,
+                                sigma=1e-3) for r in range(Nd)]
+        for r in range(Nd):
+            buf.grads[r].view(torch.int16).copy_(torch.from_numpy(flat[r].view(np.int16)))
+        buf.step(zero.hparams(lr=1e-3, weight_decay=0.01, max_grad_norm=0.01))
+        t, ovf, ss, _, _ = oracle.zero12_step_ex(Nd, N, 0, oracle.BF16, flat, om, mm, vm, oreps,
+                                                 hp, t)
+    res = buf.result()
+    assert res["step"] == t == 2 and abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
+    assert_f32_close(f32(buf.master[0]), om, "zero3 clipped master")
+    assert_f32_close(f32(buf.exp_avg_sq[0]), vm, "zero3 clipped exp_avg_sq")
+    assert_bf16_close(u16(buf.param_shard), oreps[0], "zero3 clipped bf16 shard")
+    del buf
+    free()
+
+
 # ----------------------------------------------------------------------------- building blocks
 
 def test_building_blocks_two_pass_matches_oracle():

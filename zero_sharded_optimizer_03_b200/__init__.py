@@ -18,7 +18,7 @@ __all__ = [
     "zero_read_result", "zero_begin_step", "zero_reduce_scatter", "zero_adam_shard",
     "zero_allgather", "zero_end_step", "zero3_gather_layer", "zero_step",
     "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events",
-    "zero_test_inject_stall",
+    "zero_test_inject_stall", "zero_loss_scaler_init",
     "zero_reduce_scatter_noalloc", "ZERO_NOALLOC_MAX_WINDOW", "hparams", "ZeroBuffers",
     "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_NO_TMA",
     "ZERO_FORCE_TMA",
@@ -45,13 +45,15 @@ class zero_partition_t(ctypes.Structure):
 class zero_hparams_t(ctypes.Structure):
     _fields_ = [("lr", _dbl), ("beta1", _dbl), ("beta2", _dbl), ("eps", _dbl),
                 ("weight_decay", _dbl), ("loss_scale", _dbl), ("grad_average", _i32),
-                ("reserved", _i32)]
+                ("reserved", _i32), ("max_grad_norm", _dbl)]
 
 
 class zero_step_result_t(ctypes.Structure):
     _fields_ = [("step", _i64), ("skipped", _i64), ("overflow", _i32), ("live", _i32),
                 ("grad_sumsq", _dbl), ("pending_overflow", _i32), ("reserved", _i32),
-                ("pending_sumsq", _dbl), ("error", _i32), ("reserved2", _i32)]
+                ("pending_sumsq", _dbl), ("error", _i32), ("reserved2", _i32),
+                ("loss_scale", _dbl), ("good_steps", _i64), ("dynamic_scale", _i32),
+                ("reserved3", _i32)]
 
 
 class zero_state_t(ctypes.Structure):
@@ -105,6 +107,7 @@ def _load() -> ctypes.CDLL:
         "zero_comm_volume": ([ctypes.c_int, _dbl, ctypes.c_int], _dbl),
         "zero_profile_events": ([_P, _P], ctypes.c_int),
         "zero_test_inject_stall": ([_i64], ctypes.c_int),
+        "zero_loss_scaler_init": ([_P, _dbl, _dbl, _dbl, _i64, _P], ctypes.c_int),
         "zero_reduce_scatter_noalloc": ([_P, ctypes.c_int, ctypes.c_int, _i64, _i64,
                                          ctypes.POINTER(zero_hparams_t), _P, _P, ctypes.c_int,
                                          _P], ctypes.c_int),
@@ -138,9 +141,9 @@ def _ptrs(ptrs) -> ctypes.Array:
 
 
 def hparams(lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, loss_scale=1.0,
-            grad_average=True) -> zero_hparams_t:
+            grad_average=True, max_grad_norm=0.0) -> zero_hparams_t:
     return zero_hparams_t(lr, beta1, beta2, eps, weight_decay, loss_scale,
-                          1 if grad_average else 0, 0)
+                          1 if grad_average else 0, 0, max_grad_norm)
 
 
 # ----------------------------------------------------------------------------- entry points
@@ -198,6 +201,13 @@ def zero_reduce_scatter_noalloc(grads, dtype: int, Nd: int, lo: int, hi: int,
     zero_rs_summary_t (16 bytes) that receives the window's overflow flag and sum of squares."""
     _check(lib.zero_reduce_scatter_noalloc(_ptrs(grads), dtype, Nd, lo, hi, ctypes.byref(hp),
                                            grad_out, summary, 1 if accumulate else 0, stream))
+
+
+def zero_loss_scaler_init(ws: int, init_scale: float = 65536.0, growth_factor: float = 2.0,
+                          backoff_factor: float = 0.5, growth_interval: int = 2000,
+                          stream: int = 0) -> None:
+    _check(lib.zero_loss_scaler_init(ws, init_scale, growth_factor, backoff_factor,
+                                     growth_interval, stream))
 
 
 def zero_test_inject_stall(unit: int) -> None:

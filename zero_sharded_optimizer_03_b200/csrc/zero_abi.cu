@@ -131,6 +131,8 @@ int check_hp(const zero_hparams_t* hp) {
   if (!std::isfinite(hp->weight_decay)) return fail(ZERO_EINVAL, "weight_decay must be finite");
   if (!(hp->loss_scale > 0) || !std::isfinite(hp->loss_scale))
     return fail(ZERO_EINVAL, "loss_scale must be finite and > 0");
+  if (!(hp->max_grad_norm >= 0) || !std::isfinite(hp->max_grad_norm))
+    return fail(ZERO_EINVAL, "max_grad_norm must be finite and >= 0");
   return ZERO_OK;
 }
 
@@ -148,6 +150,8 @@ zb::Consts make_consts(const zero_hparams_t* hp, int Nd) {
   c.lr = hp->lr;
   c.b1d = hp->beta1;
   c.b2d = hp->beta2;
+  c.inv_base = hp->grad_average ? (double)Nd : 1.0;
+  c.max_norm = hp->max_grad_norm;
   return c;
 }
 
@@ -329,6 +333,10 @@ int zero_read_result(const void* ws, zero_step_result_t* out, void* stream) {
   out->pending_sumsq = h.pending_sumsq;
   out->error = h.error;
   out->reserved2 = 0;
+  out->loss_scale = h.dyn ? h.scale : 0.0;
+  out->good_steps = h.dyn ? h.good : 0;
+  out->dynamic_scale = h.dyn;
+  out->reserved3 = 0;
   return ZERO_OK;
 }
 
@@ -336,6 +344,18 @@ int zero_profile_events(void* start_event, void* stop_event) {
   g_prof_start = (cudaEvent_t)start_event;
   g_prof_stop = (cudaEvent_t)stop_event;
   return ZERO_OK;
+}
+
+int zero_loss_scaler_init(void* ws, double init_scale, double growth_factor, double backoff_factor,
+                          int64_t growth_interval, void* stream) {
+  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (!(init_scale > 0) || !std::isfinite(init_scale)) return fail(ZERO_EINVAL, "init_scale must be finite and > 0");
+  if (!(growth_factor >= 1) || !std::isfinite(growth_factor)) return fail(ZERO_EINVAL, "growth_factor must be >= 1");
+  if (!(backoff_factor > 0 && backoff_factor <= 1)) return fail(ZERO_EINVAL, "backoff_factor must be in (0, 1]");
+  if (growth_interval < 1) return fail(ZERO_EINVAL, "growth_interval must be >= 1");
+  zb::scaler_init_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(header(ws), init_scale, growth_factor, backoff_factor,
+                                                             (long long)growth_interval);
+  return check_launch("scaler_init_kernel launch");
 }
 
 int zero_test_inject_stall(int64_t unit) {
@@ -371,7 +391,9 @@ int zero_reduce_scatter(const uint16_t* const* grads, int dtype, int Nd, int64_t
   a.out = grad_out;
   a.lo = lo;
   a.hi = hi;
-  a.inv = make_consts(hp, Nd).inv;
+  const zb::Consts c = make_consts(hp, Nd);
+  a.inv = c.inv;
+  a.inv_base = c.inv_base;
   a.Nd = Nd;
   a.hdr = header(ws);
   a.part = partials(ws);
@@ -494,6 +516,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       a.lo = 0;
       a.hi = Ll;
       a.inv = c.inv;
+      a.inv_base = c.inv_base;
       a.Nd = Nd;
       a.hdr = header(ws);
       a.part = partials(ws);
@@ -547,6 +570,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       a.lo = k * B;
       a.hi = (k + 1) * B < N ? (k + 1) * B : N;
       a.inv = c.inv;
+      a.inv_base = c.inv_base;
       a.Nd = Nd;
       a.hdr = header(ws);
       a.part = partials(ws);
@@ -582,6 +606,10 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     return ZERO_OK;
   }
 
+  if (hp->max_grad_norm > 0)
+    return fail(ZERO_EINVAL,
+                "gradient clipping needs the whole gradient's norm before the update: use "
+                "ZERO_TWO_PASS (or stage 3); the fused one-pass step cannot clip");
   for (int i = 0; i < 2; ++i)
     if (!st->master[i] || !st->exp_avg[i] || !st->exp_avg_sq[i])
       return fail(ZERO_EINVAL, "ZERO_FUSED needs both state copies (master/exp_avg/exp_avg_sq [0] and [1])");

@@ -42,7 +42,11 @@ struct Header {
   int last_flag;          // overflow of the last finished step
   double last_sumsq;      // sum of squares of the last finished step
   int error;              // nonzero once a kernel gave up a bounded wait (sticky until init)
-  int unused;
+  int dyn;                // dynamic loss scaling on: the gradients carry `scale`
+  double scale;           // current loss scale (dynamic)
+  double growth, backoff; // scale factors after `interval` clean steps / after an overflow
+  long long interval;
+  long long good;         // clean steps since the last change of the scale
 };
 static_assert(sizeof(Header) <= 256, "header must fit its slot");
 
@@ -72,7 +76,49 @@ struct Consts {
   float decay;  // 1 - lr*wd
   float unused;
   double lr, b1d, b2d;  // for the step-dependent bias corrections
+  double inv_base;      // Nd (mean) or 1 (sum): the unscale factor is 1/(inv_base * loss scale)
+  double max_norm;      // global-norm clipping bound (<= 0: off)
 };
+
+// Unscale factor of the step: from the host (static loss scale) or, with dynamic loss scaling,
+// 1/(inv_base * scale) from the workspace, evaluated in double and rounded once to fp32.
+__device__ __forceinline__ float step_inv(const Consts& c, const Header* h) {
+  if (!__ldcg(&h->dyn)) return c.inv;
+  return __double2float_rn(__ddiv_rn(1.0, __dmul_rn(c.inv_base, __ldcg(&h->scale))));
+}
+
+// Clipping factor min(1, max_norm/(sqrt(sumsq) + 1e-6)) in double, rounded once to fp32.
+__device__ __forceinline__ float clip_coef(double max_norm, double sumsq) {
+  if (!(max_norm > 0.0)) return 1.0f;
+  double coef = __ddiv_rn(max_norm, __dadd_rn(__dsqrt_rn(sumsq), 1e-6));
+  if (coef > 1.0) coef = 1.0;
+  return __double2float_rn(coef);
+}
+
+// End of a step: bookkeeping of the counters and of the dynamic loss scale.
+__device__ __forceinline__ void end_step(Header* h, int flip) {
+  const int of = h->pending_flag;
+  h->last_flag = of;
+  h->last_sumsq = h->pending_sumsq;
+  if (!of) {
+    h->t += 1;
+    if (flip) h->live ^= 1;
+  } else {
+    h->skipped += 1;
+  }
+  if (h->dyn) {
+    if (of) {
+      h->scale = __dmul_rn(h->scale, h->backoff);
+      h->good = 0;
+    } else if (++h->good >= h->interval) {
+      const double grown = __dmul_rn(h->scale, h->growth);
+      if (grown <= 3.4028234663852886e38) h->scale = grown;  // stays finite in fp32
+      h->good = 0;
+    }
+  }
+  h->pending_flag = 0;
+  h->pending_sumsq = 0.0;
+}
 
 struct Bias {
   float step_size;  // lr / (1 - b1^t)
@@ -294,19 +340,7 @@ __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Pa
       hdr->pending_flag |= fl;
       hdr->pending_sumsq = __dadd_rn(hdr->pending_sumsq, tot);
     }
-    if (mode & kFinalize) {
-      const int of = hdr->pending_flag;
-      hdr->last_flag = of;
-      hdr->last_sumsq = hdr->pending_sumsq;
-      if (!of) {
-        hdr->t += 1;
-        if (mode & kFlip) hdr->live ^= 1;
-      } else {
-        hdr->skipped += 1;
-      }
-      hdr->pending_flag = 0;
-      hdr->pending_sumsq = 0.0;
-    }
+    if (mode & kFinalize) end_step(hdr, mode & kFlip);
     hdr->done = 0u;
     __threadfence();
   }
@@ -334,13 +368,16 @@ template <int DT>
 __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   __shared__ Bias s_bias;
   __shared__ int s_live;
+  __shared__ float s_inv;
   if (threadIdx.x == 0) {
     s_bias = bias_for(a.c, __ldcg(&a.hdr->t) + 1);
     s_live = __ldcg(&a.hdr->live) & 1;
+    s_inv = step_inv(a.c, a.hdr);
   }
   __syncthreads();
   const Bias b = s_bias;
   const int live = s_live;
+  const float inv = s_inv;
   const float* __restrict__ sp = a.p[live];
   const float* __restrict__ sm = a.m[live];
   const float* __restrict__ sv = a.v[live];
@@ -361,7 +398,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     fan_in8<DT>(a.grads, a.Nd, i, s);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float g = __fmul_rn(s[k], a.c.inv);
+      const float g = __fmul_rn(s[k], inv);
       bad |= nonfinite(g);
       sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
       adam_elem(g, P[k], M[k], V[k], a.c, b);
@@ -377,7 +414,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
   }
   for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
     const int64_t i = sp8.scalar_index(a.lo, e);
-    const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), a.c.inv);
+    const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), inv);
     bad |= nonfinite(g);
     sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
     float P = sp[i], M = sm[i], V = sv[i];
@@ -397,7 +434,8 @@ struct RsArgs {
   const uint16_t* grads[kMaxNd];
   float* out;        // reduced gradient, indexed like the replicas
   int64_t lo, hi;
-  float inv;
+  float inv;         // static unscale factor
+  double inv_base;   // Nd or 1, for the dynamic loss scale
   int Nd;
   Header* hdr;
   Partial* part;
@@ -407,6 +445,14 @@ struct RsArgs {
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_constant__ RsArgs a) {
+  __shared__ float s_inv;
+  if (threadIdx.x == 0) {
+    s_inv = a.inv;
+    if (__ldcg(&a.hdr->dyn))
+      s_inv = __double2float_rn(__ddiv_rn(1.0, __dmul_rn(a.inv_base, __ldcg(&a.hdr->scale))));
+  }
+  __syncthreads();
+  const float inv = s_inv;
   double sq = 0.0;
   int bad = 0;
   float* __restrict__ out = a.out;
@@ -418,7 +464,7 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
     fan_in8<DT>(a.grads, a.Nd, i, s);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      s[k] = __fmul_rn(s[k], a.inv);
+      s[k] = __fmul_rn(s[k], inv);
       bad |= nonfinite(s[k]);
       sq = __dadd_rn(sq, __dmul_rn((double)s[k], (double)s[k]));
     }
@@ -427,7 +473,7 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
   }
   for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
     const int64_t i = sp8.scalar_index(a.lo, e);
-    const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), a.inv);
+    const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), inv);
     bad |= nonfinite(g);
     sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
     out[i] = g;
@@ -457,14 +503,17 @@ struct AdamArgs {
 __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ AdamArgs a) {
   __shared__ Bias s_bias;
   __shared__ int s_live, s_skip;
+  __shared__ float s_coef;
   if (threadIdx.x == 0) {
     s_bias = bias_for(a.c, __ldcg(&a.hdr->t) + 1);
     s_live = a.use_live ? (__ldcg(&a.hdr->live) & 1) : 0;
     s_skip = __ldcg(&a.hdr->pending_flag);
+    s_coef = clip_coef(a.c.max_norm, __ldcg(&a.hdr->pending_sumsq));
   }
   __syncthreads();
   if (!s_skip) {
     const Bias b = s_bias;
+    const float coef = s_coef;  // 1 unless the step's gradient norm is clipped
     float* __restrict__ P_ = a.p[s_live];
     float* __restrict__ M_ = a.m[s_live];
     float* __restrict__ V_ = a.v[s_live];
@@ -479,7 +528,7 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
       unpack(ld_stream(V_ + i), ld_stream(V_ + i + 4), V);
       unpack(ld_stream(G_ + i), ld_stream(G_ + i + 4), G);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) adam_elem(G[k], P[k], M[k], V[k], a.c, b);
+      for (int k = 0; k < 8; ++k) adam_elem(__fmul_rn(G[k], coef), P[k], M[k], V[k], a.c, b);
       st_stream(P_ + i, make_float4(P[0], P[1], P[2], P[3]));
       st_stream(P_ + i + 4, make_float4(P[4], P[5], P[6], P[7]));
       st_stream(M_ + i, make_float4(M[0], M[1], M[2], M[3]));
@@ -495,7 +544,7 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
     for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
       const int64_t i = sp8.scalar_index(a.lo, e);
       float P = P_[i], M = M_[i], V = V_[i];
-      adam_elem(G_[i], P, M, V, a.c, b);
+      adam_elem(__fmul_rn(G_[i], coef), P, M, V, a.c, b);
       P_[i] = P;
       M_[i] = M;
       V_[i] = V;
@@ -611,22 +660,30 @@ __global__ void ws_ctl_kernel(Header* h, int op, long long t0) {
     h->last_flag = 0;
     h->last_sumsq = 0.0;
     h->error = 0;
+    h->dyn = 0;
+    h->scale = 1.0;
+    h->growth = 1.0;
+    h->backoff = 1.0;
+    h->interval = 1;
+    h->good = 0;
   }
   if (op == kWsInit || op == kWsBegin) {
     h->pending_flag = 0;
     h->pending_sumsq = 0.0;
   }
-  if (op == kWsEnd) {
-    const int of = h->pending_flag;
-    h->last_flag = of;
-    h->last_sumsq = h->pending_sumsq;
-    if (!of)
-      h->t += 1;
-    else
-      h->skipped += 1;
-    h->pending_flag = 0;
-    h->pending_sumsq = 0.0;
-  }
+  if (op == kWsEnd) end_step(h, 0);
+  __threadfence();
+}
+
+// Turns on dynamic loss scaling in the workspace.
+__global__ void scaler_init_kernel(Header* h, double scale, double growth, double backoff, long long interval) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  h->dyn = 1;
+  h->scale = scale;
+  h->growth = growth;
+  h->backoff = backoff;
+  h->interval = interval;
+  h->good = 0;
   __threadfence();
 }
 

@@ -182,12 +182,14 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOffset);
   __shared__ Bias s_bias;
   __shared__ int s_live;
+  __shared__ float s_inv;
   __shared__ volatile int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     s_bias = bias_for(a.c, __ldcg(&a.hdr->t) + 1);
     s_live = __ldcg(&a.hdr->live) & 1;
+    s_inv = step_inv(a.c, a.hdr);
     s_abort = (smem_u32(smem) & 127u) ? 1 : 0;  // bulk copies need aligned buffers: never start misaligned
     for (int k = 0; k < kNumBars; ++k) mbar_init(smem_u32(&bars[k]), 1);
     fence_barrier_init();
@@ -195,6 +197,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
   __syncthreads();
   const Bias b = s_bias;
   const int live = s_live;
+  const float inv = s_inv;
   // full[s]: loads landed; empty[s]: consumers done with input stage s;
   // out_full[o]: results written to output buffer o; out_free[o]: its stores have read it
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
       if (t == 0) mbar_arrive(empty_bar(s));
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float g = __fmul_rn(acc[k], a.c.inv);
+        const float g = __fmul_rn(acc[k], inv);
         bad |= nonfinite(g);
         sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
         adam_elem(g, P[k], M[k], V[k], a.c, b);
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
       const int64_t nrest = nhead + (a.hi - tail_lo);
       for (int64_t e = (int64_t)blockIdx.x * kConsumers + t; e < nrest; e += (int64_t)gridDim.x * kConsumers) {
         const int64_t i = e < nhead ? a.lo + e : tail_lo + (e - nhead);
-        const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), a.c.inv);
+        const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), inv);
         bad |= nonfinite(g);
         sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
         float P = sp[i], M = sm[i], V = sv[i];
