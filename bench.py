@@ -58,6 +58,13 @@ WORKLOADS = {
              "with m,v prefilled",
         stage=2, Nd=64, N=1 << 28, bucket=0, gdt="bf16", sigma=1e-3, kind="heavy", t0=999,
         hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
+    "zero2-offload-gpt2-small": dict(
+        desc="ZeRO-Offload: N=124,439,808 (GPT-2 small), Nd=8, bf16 grads ~N(0,1e-3); "
+             "reduce-scatter on the GPU, AdamW (lr 6e-4 wd 0.01) on fp32 state in pinned host "
+             "memory, bf16 weights back to 8 replicas, 16M-element chunks",
+        stage=2, offload=True, chunk=1 << 24, Nd=8, N=124_439_808, bucket=0, gdt="bf16",
+        sigma=1e-3, kind="normal",
+        hp=dict(lr=6e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
     "zero3-llama7b": dict(
         desc="ZeRO-3 Llama-7B-shaped: 32 layers of q,k,v,o 4096x4096 + gate,up,down 4096x11008 "
              "(202,375,168 each), Nd=8; per layer gather from 8 bf16 shards and reduce-scatter "
@@ -222,6 +229,76 @@ def whole_job_rate(units_per_rank, world, ms_per_step):
     return world * units_per_rank / (ms_per_step / 1e3)
 
 
+# ----------------------------------------------------------------------------- offload
+
+def run_offload(args, w, world, rank, dist, dev, config):
+    """ZeRO-Offload step: reduce-scatter on the GPU, AdamW on host memory, weights back."""
+    import numpy as np
+    import torch
+
+    import synth
+    import zero_sharded_optimizer_03_b200 as zero
+    Nd, N = w["Nd"], w["N"]
+    steps = min(args.steps, 20)  # host-bound steps of ~0.1 s: keep the timed region short
+    s = torch.cuda.current_stream()
+    sp = s.cuda_stream
+    buf = zero.ZeroOffloadBuffers(Nd, N, chunk=w["chunk"], host_threads=0)
+    buf.master.numpy()[:] = synth.fill_host(synth.NORMAL, synth.F32, synth.SEED,
+                                            synth.MASTER_STREAM, N, sigma=0.02)
+    buf.init_workspace(0)
+    buf.sync_params_from_master()
+    for r in range(Nd):
+        synth.fill_device(buf.grads[r].data_ptr(), synth.NORMAL, synth.BF16, synth.SEED,
+                          synth.grad_stream(1, r), N, w["sigma"], cuda_stream=sp)
+    hp = zero.hparams(**w["hp"])
+    for _ in range(args.warmup):
+        buf.step(hp)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall = time.perf_counter()
+    t0.record(s)
+    for _ in range(steps):
+        buf.step(hp)
+    t1.record(s)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall
+    ms_total = max_over_ranks([t0.elapsed_time(t1)], dist, dev)[0]
+    res = buf.result()
+    assert res["overflow"] == 0 and res["skipped"] == 0, res
+    ms = ms_total / steps
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, times = cpu_baseline(w)
+        cpu = {"value": n / times[0], "unit": "params/s", "cores": 1, "kind": "oracle",
+               "sample": "first %d of %d parameters, Nd=%d, one ZeRO step (%.1f s)"
+               % (n, N, Nd, times[0])}
+    host_bytes = 30 * N  # grad 4 read, master/m/v 12 read + 12 written, bf16 weights 2 written
+    pcie_bytes = 6 * N   # fp32 gradient down (4), bf16 weights up (2)
+    if rank == 0:
+        config["path"] = "offload"
+        config["kernel"] = "reduce_scatter_kernel + host AdamW + gather_layer_kernel"
+        config["host_threads"] = os.cpu_count()
+        line = {"metric": METRIC, "value": whole_job_rate(N, world, ms), "unit": "params/s",
+                "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic", "config": config,
+                "roofline": {"bound": "host", "achieved": host_bytes / (ms / 1e3) / 1e9,
+                             "peak": None, "unit": "GB/s", "frac": None, "traffic": None,
+                             "pcie_gbs": pcie_bytes / (ms / 1e3) / 1e9,
+                             "note": "host-memory and PCIe bound; no measured host peak"},
+                "cpu_baseline": cpu, "e2e": None, "clocks": None,
+                "gpu_launches": steps * (-(-N // w["chunk"]) * 2 + 1),
+                "wall_s": wall}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -300,6 +377,8 @@ def main():
     else:
         torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if w.get("offload"):
+        return run_offload(args, w, world, rank, dist, dev, config)
     s = torch.cuda.current_stream()
     sp = s.cuda_stream
 

@@ -309,6 +309,53 @@ int zero_reduce_scatter_noalloc(const uint16_t *const *grads, int dtype, int Nd,
  * clears.  Units of a CTA are numbered ceil(Nd/8) gradient chunks then one state unit per tile. */
 int zero_test_inject_stall(int64_t unit);
 
+/* ------------------------------------------------------------------ ZeRO-Offload */
+
+/* Buffers of an offloaded step ([P2] "ZeRO-Offload": optimizer state and gradients in CPU
+ * memory, the CPU updates the state, the updated weights go back to the GPU).  Device: the Nd
+ * gradient and weight replicas (N elements each), an fp32 staging buffer for the reduced
+ * gradient and a bf16 staging buffer for the new weights (N elements each), the workspace.
+ * Host: the fp32 master / exp_avg / exp_avg_sq (N elements each; any host memory), and pinned
+ * (page-locked) fp32 gradient and bf16 weight buffers (N elements each) for the copies. */
+typedef struct {
+    int32_t grad_dtype;   /* ZERO_BF16 or ZERO_FP16 */
+    int32_t host_threads; /* CPU threads for the host update (0: all hardware threads) */
+    const uint16_t *grads[ZERO_MAX_ND];
+    uint16_t *params[ZERO_MAX_ND];
+    float *grad_dev;
+    uint16_t *param_dev;
+    float *grad_host;
+    uint16_t *param_host;
+    float *master_host;
+    float *exp_avg_host;
+    float *exp_avg_sq_host;
+    void *workspace;
+    void *upload_stream;  /* cudaStream_t for host->device copies and the fan-out (NULL: `stream`) */
+} zero_offload_state_t;
+
+/* AdamW on host memory (the CPU half of ZeRO-Offload).  For i < n, with g = grad[i] * clip_coef,
+ * the rule of zero_adam_shard at step t (t >= 1: the update being made), in fp32 with the same
+ * operation order, so results are bit-identical to the device kernels; param_out[i] =
+ * bf16(master[i]) when param_out is not NULL.  clip_coef in (0, 1] (1: no clipping).  Runs
+ * on `nthreads` CPU threads (0: all hardware threads) of a pool kept by the library; blocks
+ * until done.  Host pointers only. */
+int zero_host_adam(float *master, float *exp_avg, float *exp_avg_sq, const float *grad, int64_t n,
+                   const zero_hparams_t *hp, int64_t t, float clip_coef, uint16_t *param_out,
+                   int nthreads);
+
+/* One ZeRO-Offload step (stages 1/2 arithmetic, state on the host).  In chunks of `chunk`
+ * elements (0: one chunk): the device reduce-scatters the replicas into grad_dev (unscale,
+ * overflow flag, sum of squares, dynamic loss scale as in zero_step) and copies each chunk to
+ * grad_host on `stream`; once all chunks are reduced the call reads the overflow flag; unless it
+ * is set, each chunk is updated on the CPU as soon as it has landed (zero_host_adam, with the
+ * clipping factor of hp->max_grad_norm), copied to param_dev and fanned out to the Nd replicas
+ * on upload_stream, so copies in both directions overlap the CPU work; finally `stream` waits
+ * for the uploads and the step ends on the device (t, skip count, loss scale).  An overflow
+ * skips the update: host state and replicas keep their values.  Blocks the calling thread for
+ * the CPU part; device work stays queued on the streams. */
+int zero_offload_step(int Nd, int64_t N, int64_t chunk, const zero_offload_state_t *st,
+                      const zero_hparams_t *hp, void *stream);
+
 /* ------------------------------------------------------------------ accounting (host only) */
 
 /* Per-GPU model-state memory ([P1] §二 code: bytes_per_param for the 16-bit weights and again

@@ -125,3 +125,18 @@ def test_fused_step_refuses_clipping(zero):
     with pytest.raises(zero.ZeroError) as e:
         zero.zero_step(1, 4, 1000, 0, st, zero.hparams(1e-3, max_grad_norm=1.0))
     assert e.value.code == zero.ZERO_EINVAL and "ZERO_TWO_PASS" in str(e.value)
+
+
+def test_offload_step_validates_before_touching_the_device(zero):
+    hp = zero.hparams(1e-3)
+    st = zero.zero_offload_state_t()
+    cases = [(0, 10, 0, st, hp), (4, -1, 0, st, hp), (4, 10, -1, st, hp), (4, 10, 0, st, hp),
+             (4, 10, 0, st, zero.hparams(1e-3, eps=-1.0))]
+    for args in cases:
+        with pytest.raises(zero.ZeroError) as e:
+            zero.zero_offload_step(*args)
+        assert e.value.code == zero.ZERO_EINVAL
+    st.workspace = 4096  # fake: the missing staging buffers are refused first
+    with pytest.raises(zero.ZeroError) as e:
+        zero.zero_offload_step(4, 10, 0, st, hp)
+    assert "grad_dev" in str(e.value)

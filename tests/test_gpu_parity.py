@@ -435,6 +435,54 @@ def test_clipping_zero3_matches_flat_oracle():
     free()
 
 
+# ----------------------------------------------------------------------------- ZeRO-Offload
+
+@pytest.mark.parametrize("gdt,dynamic,max_norm", [(zero.ZERO_BF16, False, 0.0),
+                                                  (zero.ZERO_FP16, True, 0.05)])
+def test_offload_step_matches_oracle(gdt, dynamic, max_norm):
+    """Reduce-scatter on the GPU, AdamW on host memory, weights back to every replica: host
+    state and device replicas equal the oracle's; an overflow on step 2 is skipped."""
+    Nd, N, chunk = 4, 1_000_003, 300_000
+    odt, sdt = DT[gdt]
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=1.0, max_grad_norm=max_norm,
+              dynamic_scale=dynamic, scale_interval=2)
+    buf = zero.ZeroOffloadBuffers(Nd, N, grad_dtype=gdt, chunk=chunk, host_threads=4)
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    buf.master.copy_(torch.from_numpy(om[:N]))
+    buf.init_workspace(0)
+    if dynamic:
+        zero.zero_loss_scaler_init(buf.ws.data_ptr(), 512.0, 2.0, 0.5, 2, stream())
+    buf.sync_params_from_master()
+    oreps = [oracle.f32_to_bf16(om[:N]) for _ in range(Nd)]
+    t, scale, good = 0, 512.0, 0
+    for k in (1, 2, 3, 4):
+        sigma = float(np.float32(1e-4 * scale)) if dynamic else 1e-3
+        hg = [synth.fill_host(synth.NORMAL, sdt, SEED, synth.grad_stream(k, r), N, sigma=sigma)
+              for r in range(Nd)]
+        for r in range(Nd):
+            fill(buf.grads[r], synth.NORMAL, sdt, synth.grad_stream(k, r), sigma=sigma)
+        if k == 2:
+            bits = 0x7C00 if sdt == synth.FP16 else 0x7F80
+            put_bits(buf.grads[1], N - 3, bits)
+            hg[1][N - 3] = bits
+        buf.step(zero.hparams(lr=1e-3, weight_decay=0.01, max_grad_norm=max_norm))
+        t, ovf, ss, scale, good = oracle.zero12_step_ex(Nd, N, 0, odt, hg, om, mm, vm, oreps, hp,
+                                                        t, scale, good)
+        res = buf.result()
+        assert res["overflow"] == ovf == (1 if k == 2 else 0) and res["step"] == t
+        if dynamic:
+            assert res["loss_scale"] == scale
+    torch.cuda.synchronize()
+    assert_f32_close(buf.master.numpy(), om[:N], "offload master")
+    assert_f32_close(buf.exp_avg.numpy(), mm[:N], "offload exp_avg")
+    assert_f32_close(buf.exp_avg_sq.numpy(), vm[:N], "offload exp_avg_sq")
+    for r in range(Nd):
+        assert_bf16_close(u16(buf.params[r]), oreps[r], "offload replica %d" % r)
+    del buf
+    free()
+
+
 # ----------------------------------------------------------------------------- building blocks
 
 def test_building_blocks_two_pass_matches_oracle():

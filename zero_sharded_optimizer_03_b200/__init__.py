@@ -18,7 +18,8 @@ __all__ = [
     "zero_read_result", "zero_begin_step", "zero_reduce_scatter", "zero_adam_shard",
     "zero_allgather", "zero_end_step", "zero3_gather_layer", "zero_step",
     "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events",
-    "zero_test_inject_stall", "zero_loss_scaler_init",
+    "zero_test_inject_stall", "zero_loss_scaler_init", "zero_host_adam", "zero_offload_step",
+    "ZeroOffloadBuffers",
     "zero_reduce_scatter_noalloc", "ZERO_NOALLOC_MAX_WINDOW", "hparams", "ZeroBuffers",
     "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_NO_TMA",
     "ZERO_FORCE_TMA",
@@ -73,6 +74,14 @@ ZERO_NOALLOC_MAX_CTAS = 16384
 ZERO_NOALLOC_MAX_WINDOW = ZERO_NOALLOC_MAX_CTAS * 2048
 
 
+class zero_offload_state_t(ctypes.Structure):
+    _fields_ = [("grad_dtype", _i32), ("host_threads", _i32),
+                ("grads", _P * ZERO_MAX_ND), ("params", _P * ZERO_MAX_ND),
+                ("grad_dev", _P), ("param_dev", _P), ("grad_host", _P), ("param_host", _P),
+                ("master_host", _P), ("exp_avg_host", _P), ("exp_avg_sq_host", _P),
+                ("workspace", _P), ("upload_stream", _P)]
+
+
 class zero_mem_t(ctypes.Structure):
     _fields_ = [("optimizer_states", _dbl), ("gradients", _dbl), ("parameters", _dbl),
                 ("total", _dbl)]
@@ -108,6 +117,10 @@ def _load() -> ctypes.CDLL:
         "zero_profile_events": ([_P, _P], ctypes.c_int),
         "zero_test_inject_stall": ([_i64], ctypes.c_int),
         "zero_loss_scaler_init": ([_P, _dbl, _dbl, _dbl, _i64, _P], ctypes.c_int),
+        "zero_host_adam": ([_P, _P, _P, _P, _i64, ctypes.POINTER(zero_hparams_t), _i64,
+                            ctypes.c_float, _P, ctypes.c_int], ctypes.c_int),
+        "zero_offload_step": ([ctypes.c_int, _i64, _i64, ctypes.POINTER(zero_offload_state_t),
+                               ctypes.POINTER(zero_hparams_t), _P], ctypes.c_int),
         "zero_reduce_scatter_noalloc": ([_P, ctypes.c_int, ctypes.c_int, _i64, _i64,
                                          ctypes.POINTER(zero_hparams_t), _P, _P, ctypes.c_int,
                                          _P], ctypes.c_int),
@@ -201,6 +214,19 @@ def zero_reduce_scatter_noalloc(grads, dtype: int, Nd: int, lo: int, hi: int,
     zero_rs_summary_t (16 bytes) that receives the window's overflow flag and sum of squares."""
     _check(lib.zero_reduce_scatter_noalloc(_ptrs(grads), dtype, Nd, lo, hi, ctypes.byref(hp),
                                            grad_out, summary, 1 if accumulate else 0, stream))
+
+
+def zero_host_adam(master: int, exp_avg: int, exp_avg_sq: int, grad: int, n: int,
+                   hp: zero_hparams_t, t: int, clip_coef: float = 1.0,
+                   param_out: int | None = None, nthreads: int = 0) -> None:
+    """AdamW on host memory (pointers into host arrays), bit-identical to the device kernels."""
+    _check(lib.zero_host_adam(master, exp_avg, exp_avg_sq, grad, n, ctypes.byref(hp), t,
+                              clip_coef, param_out, nthreads))
+
+
+def zero_offload_step(Nd: int, N: int, chunk: int, state: zero_offload_state_t,
+                      hp: zero_hparams_t, stream: int = 0) -> None:
+    _check(lib.zero_offload_step(Nd, N, chunk, ctypes.byref(state), ctypes.byref(hp), stream))
 
 
 def zero_loss_scaler_init(ws: int, init_scale: float = 65536.0, growth_factor: float = 2.0,
@@ -346,3 +372,64 @@ class ZeroBuffers:
         else:
             zero_allgather(self.master[0].data_ptr(), [self.param_shard.data_ptr()], 1, 0,
                            self.Np, ZERO_GATE_ALWAYS, None, self.stream())
+
+
+class ZeroOffloadBuffers:
+    """Caller-owned buffers of a ZeRO-Offload job, allocated with torch: the Nd device gradient
+    and weight replicas, device staging buffers, pinned host staging buffers and the fp32
+    optimizer state in (pinned) host memory."""
+
+    def __init__(self, Nd: int, N: int, grad_dtype: int = ZERO_BF16, chunk: int = 1 << 24,
+                 host_threads: int = 0, device: str = "cuda"):
+        import torch
+        self.torch = torch
+        self.Nd, self.N, self.chunk = Nd, N, chunk
+        gdt = torch.bfloat16 if grad_dtype == ZERO_BF16 else torch.float16
+        n = max(N, 1)
+        self.ws = torch.zeros(zero_workspace_bytes(), dtype=torch.uint8, device=device)
+        self.grads = [torch.zeros(n, dtype=gdt, device=device) for _ in range(Nd)]
+        self.params = [torch.zeros(n, dtype=torch.bfloat16, device=device) for _ in range(Nd)]
+        self.grad_dev = torch.zeros(n, dtype=torch.float32, device=device)
+        self.param_dev = torch.zeros(n, dtype=torch.bfloat16, device=device)
+        pin = dict(pin_memory=True)
+        self.grad_host = torch.zeros(n, dtype=torch.float32, **pin)
+        self.param_host = torch.zeros(n, dtype=torch.bfloat16, **pin)
+        self.master = torch.zeros(n, dtype=torch.float32, **pin)
+        self.exp_avg = torch.zeros(n, dtype=torch.float32, **pin)
+        self.exp_avg_sq = torch.zeros(n, dtype=torch.float32, **pin)
+        self.upload = torch.cuda.Stream()
+        st = zero_offload_state_t()
+        st.grad_dtype = grad_dtype
+        st.host_threads = host_threads
+        for r in range(Nd):
+            st.grads[r] = self.grads[r].data_ptr()
+            st.params[r] = self.params[r].data_ptr()
+        st.grad_dev = self.grad_dev.data_ptr()
+        st.param_dev = self.param_dev.data_ptr()
+        st.grad_host = self.grad_host.data_ptr()
+        st.param_host = self.param_host.data_ptr()
+        st.master_host = self.master.data_ptr()
+        st.exp_avg_host = self.exp_avg.data_ptr()
+        st.exp_avg_sq_host = self.exp_avg_sq.data_ptr()
+        st.workspace = self.ws.data_ptr()
+        st.upload_stream = self.upload.cuda_stream
+        self.state = st
+
+    def stream(self) -> int:
+        return self.torch.cuda.current_stream().cuda_stream
+
+    def init_workspace(self, t: int = 0) -> None:
+        zero_workspace_init(self.ws.data_ptr(), t, self.stream())
+
+    def sync_params_from_master(self) -> None:
+        """Upload bf16(master) into every device weight replica (the initial all-gather)."""
+        staging = self.master.to(self.grad_dev.device, non_blocking=False)
+        zero_allgather(staging.data_ptr(), [p.data_ptr() for p in self.params], self.Nd, 0,
+                       self.N, ZERO_GATE_ALWAYS, None, self.stream())
+        self.torch.cuda.current_stream().synchronize()
+
+    def step(self, hp: zero_hparams_t) -> None:
+        zero_offload_step(self.Nd, self.N, self.chunk, self.state, hp, self.stream())
+
+    def result(self) -> dict:
+        return zero_read_result(self.ws.data_ptr(), self.stream())

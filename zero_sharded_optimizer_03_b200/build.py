@@ -15,14 +15,14 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libzero.so")
-SOURCES = ["zero_abi.cu", "zero_accounting.cpp"]
-DEPS = SOURCES + ["zero_kernels.cuh"]
+SOURCES = ["zero_abi.cu", "zero_accounting.cpp", "zero_host_adam.cpp"]
+DEPS = SOURCES + ["zero_kernels.cuh", "zero_tma.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
     "-fmad=false",                      # every fp32/fp64 operation rounds on its own
-    "-Xcompiler", "-fPIC,-ffp-contract=off",
+    "-Xcompiler", "-fPIC,-ffp-contract=off,-fno-math-errno",
     "-Xptxas", "-v",
     "-shared",
 ]

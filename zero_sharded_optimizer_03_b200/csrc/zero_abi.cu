@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "zero.h"
 #include "zero_kernels.cuh"
@@ -284,6 +285,14 @@ int do_gather(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* const*
 }
 
 }  // namespace
+
+int zero_internal_fail(int code, const char* msg) { return fail(code, "%s", msg); }
+
+namespace zh {  // zero_host_adam.cpp
+void adam_host(float* p, float* m, float* v, const float* g, uint16_t* out16, int64_t n, const zero_hparams_t* hp,
+               int64_t t, float coef, int nthreads);
+float clip_factor(double max_norm, double sumsq);
+}  // namespace zh
 
 // ==================================================================== C ABI
 
@@ -867,4 +876,107 @@ extern "C" int zero_reduce_scatter_noalloc(const uint16_t* const* grads, int dty
   else
     reduce_scatter_noalloc_kernel<0><<<(unsigned)grid, zb::kThreads, 0, s>>>(a);
   return check_launch("reduce_scatter_noalloc_kernel launch");
+}
+
+// ==================================================================== ZeRO-Offload step
+
+namespace {
+
+struct EventRing {  // per-chunk completion events, destroyed on every exit path
+  std::vector<cudaEvent_t> ev;
+  ~EventRing() {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);
+  }
+};
+
+}  // namespace
+
+extern "C" int zero_offload_step(int Nd, int64_t N, int64_t chunk, const zero_offload_state_t* st,
+                                 const zero_hparams_t* hp, void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if ((rc = check_hp(hp))) return rc;
+  if (!st) return fail(ZERO_EINVAL, "state is NULL");
+  if (N < 0 || chunk < 0) return fail(ZERO_EINVAL, "N and chunk must be >= 0");
+  if (st->grad_dtype != ZERO_BF16 && st->grad_dtype != ZERO_FP16) return fail(ZERO_EINVAL, "grad_dtype=%d", st->grad_dtype);
+  if (!st->workspace) return fail(ZERO_EINVAL, "workspace is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  void* ws = st->workspace;
+  if (N == 0) return launch_ws(ws, zb::kWsEnd, 0, s);
+  if (!st->grad_dev || !st->param_dev || !st->grad_host || !st->param_host || !st->master_host ||
+      !st->exp_avg_host || !st->exp_avg_sq_host)
+    return fail(ZERO_EINVAL, "offload state needs grad_dev, param_dev, grad_host, param_host and the host fp32 state");
+  bool al = aligned16(st->grad_dev) && aligned16(st->param_dev);
+  if ((rc = check_ptrs(st->grads, Nd, "grads", &al))) return rc;
+  if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
+  cudaStream_t up = st->upload_stream ? (cudaStream_t)st->upload_stream : s;
+  const zb::Consts c = make_consts(hp, Nd);
+  const int64_t C = chunk > 0 ? chunk : N;
+  const int64_t nc = (N + C - 1) / C;
+  EventRing ring;
+  ring.ev.assign((size_t)nc + 2, nullptr);
+  for (auto& e : ring.ev) {
+    cudaError_t e2 = cudaEventCreateWithFlags(&e, cudaEventDisableTiming);
+    if (e2 != cudaSuccess) return cuda_fail(e2, "cudaEventCreateWithFlags");
+  }
+  cudaEvent_t ev_rs = ring.ev[nc], ev_up = ring.ev[nc + 1];
+  prof_mark(true, s);
+  // 1. reduce-scatter every chunk into the fp32 staging buffer (overflow flag and norm
+  //    accumulate in the workspace), then stream the chunks to host memory
+  for (int64_t k = 0; k < nc; ++k) {
+    zb::RsArgs a;
+    std::memset(&a, 0, sizeof a);
+    for (int r = 0; r < Nd; ++r) a.grads[r] = st->grads[r];
+    a.out = st->grad_dev;
+    a.lo = k * C;
+    a.hi = (k + 1) * C < N ? (k + 1) * C : N;
+    a.inv = c.inv;
+    a.inv_base = c.inv_base;
+    a.Nd = Nd;
+    a.hdr = header(ws);
+    a.part = partials(ws);
+    a.mode = k == 0 ? zb::kAccSet : zb::kAccAdd;
+    a.vec = al;
+    if ((rc = launch_rs(st->grad_dtype, a, s))) return rc;
+  }
+  cudaError_t e = cudaEventRecord(ev_rs, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  for (int64_t k = 0; k < nc; ++k) {
+    const int64_t lo = k * C, len = (k + 1) * C < N ? C : N - lo;
+    e = cudaMemcpyAsync(st->grad_host + lo, st->grad_dev + lo, (size_t)len * 4, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(gradient to host)");
+    if ((e = cudaEventRecord(ring.ev[k], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
+  // 2. the overflow decision and the norm, once every chunk is reduced
+  if ((e = cudaEventSynchronize(ev_rs)) != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+  zb::Header h;
+  if ((e = cudaMemcpyAsync(&h, ws, sizeof h, cudaMemcpyDeviceToHost, up)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpyAsync(workspace)");
+  if ((e = cudaStreamSynchronize(up)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  if (!h.pending_flag) {
+    // 3. host AdamW chunk by chunk as the gradients land; each chunk's bf16 weights go back
+    //    and are fanned out to the Nd replicas on the upload stream, overlapping the next chunk
+    const float coef = zh::clip_factor(hp->max_grad_norm, h.pending_sumsq);
+    for (int64_t k = 0; k < nc; ++k) {
+      const int64_t lo = k * C, len = (k + 1) * C < N ? C : N - lo;
+      if ((e = cudaEventSynchronize(ring.ev[k])) != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+      zh::adam_host(st->master_host + lo, st->exp_avg_host + lo, st->exp_avg_sq_host + lo, st->grad_host + lo,
+                    st->param_host + lo, len, hp, h.t + 1, coef, st->host_threads);
+      e = cudaMemcpyAsync(st->param_dev + lo, st->param_host + lo, (size_t)len * 2, cudaMemcpyHostToDevice, up);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(weights to device)");
+      const uint16_t* src[1] = {st->param_dev + lo};
+      uint16_t* dst[ZERO_MAX_ND];
+      for (int r = 0; r < Nd; ++r) dst[r] = st->params[r] + lo;
+      if ((rc = do_gather(src, 1, len, dst, Nd, up))) return rc;
+    }
+  }
+  if ((e = cudaEventRecord(ev_up, up)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = cudaStreamWaitEvent(s, ev_up, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  prof_mark(false, s);
+  // 4. end of step on the device: t, skip count and the dynamic loss scale
+  rc = launch_ws(ws, zb::kWsEnd, 0, s);
+  if (rc) return rc;
+  // the events may be destroyed now: pending work that refers to them still completes
+  return ZERO_OK;
 }
