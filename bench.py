@@ -321,6 +321,8 @@ def main():
                     help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather")
     ap.add_argument("--bucket-override", type=int, default=-1,
                     help="stages 1/2: run with a different bucket size (0 = one bucket)")
+    ap.add_argument("--layer-override", type=int, default=0,
+                    help="stage 3: run with a different layer length")
     ap.add_argument("--n-override", type=int, default=0,
                     help="run the workload at a different N (small cases for profiling)")
     args = ap.parse_args()
@@ -329,6 +331,9 @@ def main():
     if args.n_override:
         w["N"] = args.n_override
         w["desc"] += " [N overridden to %d]" % args.n_override
+    if args.layer_override and w["stage"] == 3:
+        w["layer"] = w["bucket"] = args.layer_override
+        w["desc"] += " [layer overridden to %d]" % args.layer_override
     if args.bucket_override >= 0 and w["stage"] != 3:
         w["bucket"] = args.bucket_override
         w["desc"] += " [bucket overridden to %d]" % args.bucket_override

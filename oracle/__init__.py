@@ -283,13 +283,14 @@ def clip_coef(sumsq: float, max_norm: float) -> float:
 def _hpx(hp: dict) -> np.ndarray:
     return np.concatenate([_hp(hp), np.array(
         [hp.get("max_grad_norm", 0.0), hp.get("scale_growth", 2.0), hp.get("scale_backoff", 0.5),
-         float(hp.get("scale_interval", 2000)), 1.0 if hp.get("dynamic_scale", False) else 0.0],
-        dtype=np.float64)])
+         float(hp.get("scale_interval", 2000)), 1.0 if hp.get("dynamic_scale", False) else 0.0,
+         1.0 if hp.get("bf16_grad", False) else 0.0], dtype=np.float64)])
 
 
 def zero12_step_ex(Nd, N, bucket, dtype, grads, master, m, v, replicas, hp, t, scale=None, good=0):
-    """ZeRO-1/2 step with clipping (hp['max_grad_norm']) and, if hp['dynamic_scale'], the
-    dynamic loss scale `scale` / `good`.  Returns (t, overflow, sumsq, scale, good)."""
+    """ZeRO-1/2 step with clipping (hp['max_grad_norm']), the bf16-kept reduced gradient
+    (hp['bf16_grad']) and, if hp['dynamic_scale'], the dynamic loss scale `scale` / `good`.
+    Returns (t, overflow, sumsq, scale, good)."""
     tt = ctypes.c_int64(t)
     ovf = ctypes.c_int(0)
     ss = ctypes.c_double(0.0)

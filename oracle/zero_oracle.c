@@ -499,14 +499,44 @@ float oracle_clip_coef(double sumsq, double max_norm)
     return (float)coef;
 }
 
-/* ZeRO-1/2 step with the two extensions.  hpx = {lr, beta1, beta2, eps, weight_decay,
- * loss_scale, grad_average, max_grad_norm, growth, backoff, interval, dynamic}.  With dynamic
+/* Reduce-scatter whose result is kept as bf16 (16-bit gradient partitions, a memory-saving
+ * variant the pages do not describe; reading: the reduced fp32 mean is rounded to bf16, nearest
+ * even, and the overflow check, the sum of squares and the update all use the rounded value).
+ * `out` receives the rounded values widened back to fp32. */
+void oracle_reduce_scatter_window_bf16(int Nd, int64_t N, int dtype, const uint16_t *const *grads,
+                                       float inv, int64_t lo, int64_t hi, float *out, int *overflow,
+                                       double *sumsq)
+{
+    int64_t part[3];
+    oracle_partition(N, Nd, part);
+    int64_t S = part[0];
+    for (int r = 0; r < Nd; r++) {
+        for (int64_t k = 0; k < S; k++) {
+            int64_t i = (int64_t)r * S + k;
+            if (i < lo || i >= hi) continue;
+            if (i >= N) {
+                out[i] = 0.0f;
+                continue;
+            }
+            float s = 0.0f;
+            for (int q = 0; q < Nd; q++) s = s + grad_value(grads[q], i, dtype);
+            float g = oracle_bf16_to_f32(oracle_f32_to_bf16(s * inv));
+            out[i] = g;
+            if (!isfinite(g)) *overflow = 1;
+            *sumsq += (double)g * (double)g;
+        }
+    }
+}
+
+/* ZeRO-1/2 step with the extensions.  hpx = {lr, beta1, beta2, eps, weight_decay,
+ * loss_scale, grad_average, max_grad_norm, growth, backoff, interval, dynamic, bf16_grad}
+ * (bf16_grad != 0: the reduced gradient is kept as bf16, see above).  With dynamic
  * != 0 the gradients carry the scale *scale (updated on return, with *good) instead of
  * hpx[5].  Order: reduce-scatter (mean, unscaled), overflow check, clipping of the reduced
  * gradient, Adam per shard, all-gather, scaler update. */
 int oracle_zero12_step_ex(int Nd, int64_t N, int64_t bucket, int dtype, const uint16_t *const *grads,
                           float *master, float *m, float *v, uint16_t *const *replicas,
-                          const double hpx[12], int64_t *t, double *scale, int64_t *good,
+                          const double hpx[13], int64_t *t, double *scale, int64_t *good,
                           int *overflow, double *sumsq)
 {
     int64_t part[3];
@@ -525,7 +555,10 @@ int oracle_zero12_step_ex(int Nd, int64_t N, int64_t bucket, int dtype, const ui
     int64_t w = bucket > 0 ? bucket : (Np > 0 ? Np : 1);
     for (int64_t lo = 0; lo < Np; lo += w) {
         int64_t hi = lo + w < Np ? lo + w : Np;
-        oracle_reduce_scatter_window(Nd, N, dtype, grads, c.inv, lo, hi, g, overflow, sumsq);
+        if (hpx[12] != 0.0)
+            oracle_reduce_scatter_window_bf16(Nd, N, dtype, grads, c.inv, lo, hi, g, overflow, sumsq);
+        else
+            oracle_reduce_scatter_window(Nd, N, dtype, grads, c.inv, lo, hi, g, overflow, sumsq);
     }
     if (!*overflow) {
         float coef = oracle_clip_coef(*sumsq, hpx[7]);

@@ -116,3 +116,24 @@ def test_dynamic_scale_equals_static_scale_and_backs_off():
         scales.append(scale)
     assert all(x.tobytes() == y.tobytes() for x, y in zip(dyn, sta))
     assert scales == [1024.0, 2048.0, 1024.0, 1024.0, 2048.0, 2048.0]
+
+
+def test_bf16_kept_gradient_equals_rounding_then_update():
+    """The bf16-kept reduced gradient variant equals: reduce-scatter (pinned), round to bf16
+    (pinned), then the pinned Adam on the rounded values, with the norm of the rounded values."""
+    Nd, N = 4, 1001
+    S, Np, _ = oracle.partition(N, Nd)
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=1.0, bf16_grad=True, max_grad_norm=0.02)
+    init = np.zeros(Np, np.float32)
+    init[:N] = synth.fill_host(synth.NORMAL, synth.F32, synth.SEED, 1, N, sigma=0.02)
+    g16 = _grads(Nd, N, synth.BF16, 1e-3)
+    p, m, v = init.copy(), np.zeros(Np, np.float32), np.zeros(Np, np.float32)
+    reps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t, ovf, ss, _, _ = oracle.zero12_step_ex(Nd, N, 0, oracle.BF16, g16, p, m, v, reps, hp, 0)
+    g, _, _ = oracle.reduce_scatter(Nd, N, oracle.BF16, g16, hp)
+    gr = oracle.bf16_to_f32(oracle.f32_to_bf16(g))
+    assert ss == float((gr[:N].astype(np.float64) ** 2).sum())
+    gr = (gr * np.float32(oracle.clip_coef(ss, 0.02))).astype(np.float32)
+    q, qm, qv = init.copy(), np.zeros(Np, np.float32), np.zeros(Np, np.float32)
+    oracle.adam(q[:N], qm[:N], qv[:N], gr[:N], hp, Nd, 1)
+    assert ovf == 0 and t == 1 and p.tobytes() == q.tobytes() and m.tobytes() == qm.tobytes()
