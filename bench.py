@@ -76,14 +76,15 @@ WORKLOADS = {
 DEFAULT = "zero1-gpt2-small"
 
 
-def bytes_per_param(w, two_pass=False) -> int:
+def bytes_per_param(w, two_pass=False, g16=False) -> int:
     Nd = w["Nd"]
+    gb = 2 if g16 else 4  # bytes of the kept reduced gradient
     if w["stage"] == 3:
-        # gather: 2 read + 2Nd written; RS: 2Nd read + 4 written; Adam + cast: 4 + 24 + 2
-        return (2 + 2 * Nd) + (2 * Nd + 4) + (4 + 24 + 2)
+        # gather: 2 read + 2Nd written; RS: 2Nd read + gb written; Adam + cast: gb + 24 + 2
+        return (2 + 2 * Nd) + (2 * Nd + gb) + (gb + 24 + 2)
     if two_pass:
-        # RS: 2Nd read + 4 written; Adam + cast + AG: 4 + 24 read/written + 2Nd written
-        return (2 * Nd + 4) + (4 + 24 + 2 * Nd)
+        # RS: 2Nd read + gb written; Adam + cast + AG: gb + 24 read/written + 2Nd written
+        return (2 * Nd + gb) + (gb + 24 + 2 * Nd)
     # fused step: Nd 2-byte gradient reads, fp32 master/m/v read + write, Nd 2-byte weight writes
     return 2 * Nd + 24 + 2 * Nd
 
@@ -317,6 +318,8 @@ def main():
                     help="fused path: always the register-pipelined kernel")
     ap.add_argument("--tma", action="store_true",
                     help="fused path: always the TMA-pipelined kernel")
+    ap.add_argument("--bf16-grad-shard", action="store_true",
+                    help="two-pass / stage 3: keep the reduced gradient as bf16")
     ap.add_argument("--two-pass", action="store_true",
                     help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather")
     ap.add_argument("--bucket-override", type=int, default=-1,
@@ -343,8 +346,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     config = {"workload": w["desc"], "N": w["N"], "Nd": w["Nd"], "stage": w["stage"],
               "bucket": w["bucket"], "grad_dtype": w["gdt"], "state_dtype": "f32",
-              "path": "two-pass" if args.two_pass else ("per-layer" if w["stage"] == 3 else
-                                                         "fused"),
+              "path": ("two-pass" if args.two_pass else ("per-layer" if w["stage"] == 3 else
+                                                          "fused"))
+              + (", bf16 gradient shard" if args.bf16_grad_shard else ""),
               "weights_dtype": "bf16", "parallelism": "replicas (%d simulated ranks per GPU)"
               % w["Nd"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
               % (2 * w["Nd"] * w["N"] / 1e9)}
@@ -408,9 +412,13 @@ def main():
     else:
         line_kernel = "fused_step_tma_kernel" if tma_path else "fused_step_kernel"
     config["kernel"] = line_kernel
+    if args.bf16_grad_shard:
+        flags |= zero.ZERO_BF16_GRAD_SHARD
     if stage == 3:
         assert w["layer"] % Nd == 0 and N % w["layer"] == 0, "unpadded layers expected"
-        buf = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, layer_len=w["layer"])
+        buf = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, layer_len=w["layer"],
+                               flags=(zero.ZERO_BF16_GRAD_SHARD if args.bf16_grad_shard else 0)
+                               | (zero.ZERO_NO_TMA if args.no_tma else 0))
     else:
         buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt, flags=flags)
     glen = buf.grads[0].numel()  # N (stages 1/2) or one layer (stage 3, reused per layer)
@@ -487,7 +495,7 @@ def main():
     ms_total, kern_ms = max_over_ranks([ms_total, kern_ms], dist, dev)
     ms_step = ms_total / args.steps
     value = whole_job_rate(N, world, ms_step)
-    bpp = bytes_per_param(w, args.two_pass)
+    bpp = bytes_per_param(w, args.two_pass, args.bf16_grad_shard)
     achieved = bpp * N / (kern_ms / 1e3) / 1e9
     peak, peak_src = peaks()
     tr = None

@@ -57,8 +57,11 @@ extern "C" {
 /* zero_step flags */
 #define ZERO_FUSED 0     /* stages 1/2: one fused pass (default); state copies ping-pong */
 #define ZERO_TWO_PASS 1  /* stages 1/2: reduce-scatter into grad_shard, then Adam + all-gather */
-#define ZERO_NO_TMA 2    /* ZERO_FUSED: always use the register-pipelined kernel */
+#define ZERO_NO_TMA 2    /* ZERO_FUSED: always use the register-pipelined kernel; stage 3: gather
+                            layers with the register kernel instead of the TMA fan-out */
 #define ZERO_FORCE_TMA 4 /* ZERO_FUSED: use the TMA-pipelined kernel whenever buffers are aligned */
+#define ZERO_BF16_GRAD_SHARD 8 /* ZERO_TWO_PASS / stage 3: keep the reduced gradient as bf16 (see
+                                  grad_shard); not described by the pages */
 
 /* zero_allgather gates */
 #define ZERO_GATE_ALWAYS 0      /* always cast and write */
@@ -130,7 +133,11 @@ typedef struct {
     float *master[2];
     float *exp_avg[2];
     float *exp_avg_sq[2];
-    float *grad_shard;      /* fp32 reduced gradient, same padded length (ZERO_TWO_PASS, stage 3) */
+    float *grad_shard;      /* reduced gradient, same padded length (ZERO_TWO_PASS, stage 3): fp32,
+                               or bf16 (uint16_t storage, cast to float*) with ZERO_BF16_GRAD_SHARD:
+                               the reduced mean is then rounded to bf16 (nearest even) before it is
+                               stored, and the overflow check, the norm and the update use the
+                               rounded value; 2 bytes per element of memory and traffic saved */
     uint16_t *param_shard;  /* stage 3: bf16 weights, the Nd shards of every layer (padded) */
     int64_t grad_layer_stride;
     int64_t param_layer_stride;

@@ -125,6 +125,10 @@ def test_fused_step_refuses_clipping(zero):
     with pytest.raises(zero.ZeroError) as e:
         zero.zero_step(1, 4, 1000, 0, st, zero.hparams(1e-3, max_grad_norm=1.0))
     assert e.value.code == zero.ZERO_EINVAL and "ZERO_TWO_PASS" in str(e.value)
+    st.flags = zero.ZERO_FUSED | zero.ZERO_BF16_GRAD_SHARD  # no gradient shard to keep
+    with pytest.raises(zero.ZeroError) as e:
+        zero.zero_step(2, 4, 1000, 0, st, zero.hparams(1e-3))
+    assert "ZERO_BF16_GRAD_SHARD" in str(e.value)
 
 
 def test_offload_step_validates_before_touching_the_device(zero):

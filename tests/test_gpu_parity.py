@@ -435,6 +435,49 @@ def test_clipping_zero3_matches_flat_oracle():
     free()
 
 
+@pytest.mark.parametrize("max_norm", [0.0, 0.01])
+def test_bf16_grad_shard_zero3_and_two_pass_match_oracle(max_norm):
+    """The reduced gradient kept as bf16: ZeRO-3 (per-layer) and the two-pass ZeRO-2 step both
+    equal the oracle's bf16-kept variant (ZeRO-3 against the flat oracle: same arithmetic)."""
+    Nd, L, nl = 4, 8192, 3
+    N = L * nl
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=1.0, max_grad_norm=max_norm, bf16_grad=True)
+    chp = zero.hparams(lr=1e-3, weight_decay=0.01, max_grad_norm=max_norm)
+    z3 = zero.ZeroBuffers(3, Nd, N, layer_len=L, per_layer_buffers=True,
+                          flags=zero.ZERO_BF16_GRAD_SHARD)
+    tp = zero.ZeroBuffers(2, Nd, N, flags=zero.ZERO_TWO_PASS | zero.ZERO_BF16_GRAD_SHARD)
+    assert z3.grad_shard.dtype == torch.bfloat16 and tp.grad_shard.dtype == torch.bfloat16
+    om = synth.fill_host(synth.NORMAL, synth.F32, SEED, synth.MASTER_STREAM, N, sigma=0.02)
+    for b in (z3, tp):
+        b.master[0].copy_(torch.from_numpy(om))
+        b.init_workspace(0)
+        b.sync_params_from_master()
+    mm = np.zeros(N, np.float32)
+    vm = np.zeros(N, np.float32)
+    oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
+    t = 0
+    for k in (1, 2):
+        flat = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(k, r), N,
+                                sigma=1e-3) for r in range(Nd)]
+        for b in (z3, tp):
+            for r in range(Nd):
+                b.grads[r].view(torch.int16).copy_(torch.from_numpy(flat[r].view(np.int16)))
+            b.step(chp)
+        t, ovf, ss, _, _ = oracle.zero12_step_ex(Nd, N, 0, oracle.BF16, flat, om, mm, vm, oreps,
+                                                 hp, t)
+    for b, tag in ((z3, "zero3"), (tp, "two-pass")):
+        res = b.result()
+        assert res["step"] == t == 2 and abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
+        assert_f32_close(f32(b.master[0]), om, tag + " bf16-grad master")
+        assert_f32_close(f32(b.exp_avg[0]), mm, tag + " bf16-grad exp_avg")
+        assert_f32_close(f32(b.exp_avg_sq[0]), vm, tag + " bf16-grad exp_avg_sq")
+    assert_bf16_close(u16(z3.param_shard), oreps[0], "zero3 bf16-grad weights")
+    for r in range(Nd):
+        assert_bf16_close(u16(tp.params[r]), oreps[r], "two-pass bf16-grad replica")
+    del z3, tp
+    free()
+
+
 # ----------------------------------------------------------------------------- ZeRO-Offload
 
 @pytest.mark.parametrize("gdt,dynamic,max_norm", [(zero.ZERO_BF16, False, 0.0),

@@ -22,7 +22,7 @@ __all__ = [
     "ZeroOffloadBuffers",
     "zero_reduce_scatter_noalloc", "ZERO_NOALLOC_MAX_WINDOW", "hparams", "ZeroBuffers",
     "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_NO_TMA",
-    "ZERO_FORCE_TMA",
+    "ZERO_FORCE_TMA", "ZERO_BF16_GRAD_SHARD",
     "ZERO_GATE_ALWAYS",
     "ZERO_GATE_NO_OVERFLOW", "ZERO_MAX_ND",
 ]
@@ -32,7 +32,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzero.so"
 ZERO_OK, ZERO_EINVAL, ZERO_ECUDA = 0, -1, -2
 ZERO_MAX_ND = 64
 ZERO_BF16, ZERO_FP16 = 0, 1
-ZERO_FUSED, ZERO_TWO_PASS, ZERO_NO_TMA, ZERO_FORCE_TMA = 0, 1, 2, 4
+ZERO_FUSED, ZERO_TWO_PASS, ZERO_NO_TMA, ZERO_FORCE_TMA, ZERO_BF16_GRAD_SHARD = 0, 1, 2, 4, 8
 ZERO_GATE_ALWAYS, ZERO_GATE_NO_OVERFLOW = 0, 1
 
 _i64, _i32, _dbl, _P = ctypes.c_int64, ctypes.c_int32, ctypes.c_double, ctypes.c_void_p
@@ -309,7 +309,9 @@ class ZeroBuffers:
             self.master = [torch.zeros(self.Np, **f32) for _ in range(copies)]
             self.exp_avg = [torch.zeros(self.Np, **f32) for _ in range(copies)]
             self.exp_avg_sq = [torch.zeros(self.Np, **f32) for _ in range(copies)]
-            self.grad_shard = torch.zeros(self.Np, **f32) if flags & ZERO_TWO_PASS else None
+            gs_dt = torch.bfloat16 if flags & ZERO_BF16_GRAD_SHARD else torch.float32
+            self.grad_shard = (torch.zeros(self.Np, dtype=gs_dt, device=device)
+                               if flags & ZERO_TWO_PASS else None)
             self.param_shard = None
         elif stage == 3:
             L = layer_len if layer_len > 0 else N
@@ -326,7 +328,8 @@ class ZeroBuffers:
             self.master = [torch.zeros(self.Np, **f32)]
             self.exp_avg = [torch.zeros(self.Np, **f32)]
             self.exp_avg_sq = [torch.zeros(self.Np, **f32)]
-            self.grad_shard = torch.zeros(self.Np, **f32)
+            gs_dt = torch.bfloat16 if flags & ZERO_BF16_GRAD_SHARD else torch.float32
+            self.grad_shard = torch.zeros(self.Np, dtype=gs_dt, device=device)
             self.param_shard = torch.zeros(self.Np, dtype=torch.bfloat16, device=device)
             st.grad_layer_stride = stride
             st.param_layer_stride = stride

@@ -37,16 +37,20 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Resident CTAs per SM for each kernel, cached per device (occupancy does not change).
 constexpr int kMaxDevices = 64;
 enum KernelId {
-  kFusedBf16, kFusedFp16, kRsBf16, kRsFp16, kAdam, kCast, kGather, kNumKernels
+  kFusedBf16, kFusedFp16, kRsBf16, kRsFp16, kRsBf16Out16, kRsFp16Out16, kAdam, kAdamG16, kCast, kGather,
+  kNumKernels
 };
 
 const void* kernel_ptr(int id) {
   switch (id) {
     case kFusedBf16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0>);
     case kFusedFp16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1>);
-    case kRsBf16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0>);
-    case kRsFp16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<1>);
-    case kAdam: return reinterpret_cast<const void*>(&zb::adam_kernel);
+    case kRsBf16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0, false>);
+    case kRsFp16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<1, false>);
+    case kRsBf16Out16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0, true>);
+    case kRsFp16Out16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<1, true>);
+    case kAdam: return reinterpret_cast<const void*>(&zb::adam_kernel<false>);
+    case kAdamG16: return reinterpret_cast<const void*>(&zb::adam_kernel<true>);
     case kCast: return reinterpret_cast<const void*>(&zb::cast_allgather_kernel);
     default: return reinterpret_cast<const void*>(&zb::gather_layer_kernel);
   }
@@ -56,6 +60,7 @@ struct DeviceInfo {
   int sms = 0;
   int per_sm[kNumKernels] = {};
   bool tma_ready = false;  // dynamic shared memory attribute set for the TMA kernels
+  int gather_tma_per_sm = 0;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -107,10 +112,23 @@ int tma_setup(int* sms) {
       e = cudaFuncSetAttribute(zb::fused_step_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)zb::kTmaSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(TMA shared memory)");
+    e = cudaFuncSetAttribute(zb::gather_layer_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)zb::kGSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(TMA gather shared memory)");
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, zb::gather_layer_tma_kernel, 32, zb::kGSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    d.gather_tma_per_sm = n > 0 ? n : 1;
     d.tma_ready = true;
   }
   *sms = d.sms;
   return ZERO_OK;
+}
+
+int gather_tma_per_sm() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+  return g_dev[dev].gather_tma_per_sm > 0 ? g_dev[dev].gather_tma_per_sm : 1;
 }
 
 int check_launch(const char* what) {
@@ -225,22 +243,31 @@ int launch_fused_tma(int dtype, zb::TmaArgs& a, cudaStream_t s) {
 }
 
 int launch_rs(int dtype, const zb::RsArgs& a, cudaStream_t s) {
-  const int kid = dtype == ZERO_FP16 ? kRsFp16 : kRsBf16;
+  const bool o16 = a.out16 != nullptr;
+  const int kid = dtype == ZERO_FP16 ? (o16 ? kRsFp16Out16 : kRsFp16) : (o16 ? kRsBf16Out16 : kRsBf16);
   int grid = 0;
   int rc = grid_for(kid, (a.hi - a.lo + 7) / 8, &grid);
   if (rc) return rc;
-  if (dtype == ZERO_FP16)
-    zb::reduce_scatter_kernel<1><<<grid, zb::kThreads, 0, s>>>(a);
+  if (dtype == ZERO_FP16 && o16)
+    zb::reduce_scatter_kernel<1, true><<<grid, zb::kThreads, 0, s>>>(a);
+  else if (dtype == ZERO_FP16)
+    zb::reduce_scatter_kernel<1, false><<<grid, zb::kThreads, 0, s>>>(a);
+  else if (o16)
+    zb::reduce_scatter_kernel<0, true><<<grid, zb::kThreads, 0, s>>>(a);
   else
-    zb::reduce_scatter_kernel<0><<<grid, zb::kThreads, 0, s>>>(a);
+    zb::reduce_scatter_kernel<0, false><<<grid, zb::kThreads, 0, s>>>(a);
   return check_launch("reduce_scatter_kernel launch");
 }
 
 int launch_adam(const zb::AdamArgs& a, cudaStream_t s) {
+  const bool g16 = a.g16 != nullptr;
   int grid = 0;
-  int rc = grid_for(kAdam, (a.hi - a.lo + 7) / 8, &grid);
+  int rc = grid_for(g16 ? kAdamG16 : kAdam, (a.hi - a.lo + 7) / 8, &grid);
   if (rc) return rc;
-  zb::adam_kernel<<<grid, zb::kThreads, 0, s>>>(a);
+  if (g16)
+    zb::adam_kernel<true><<<grid, zb::kThreads, 0, s>>>(a);
+  else
+    zb::adam_kernel<false><<<grid, zb::kThreads, 0, s>>>(a);
   return check_launch("adam_kernel launch");
 }
 
@@ -256,6 +283,11 @@ int launch_ws(void* ws, int op, long long t0, cudaStream_t s) {
   zb::ws_ctl_kernel<<<1, 32, 0, s>>>(header(ws), op, t0);
   return check_launch("ws_ctl_kernel launch");
 }
+
+// ZeRO-3 layer gather through the TMA (zero_step stage 3): needs S % 8 == 0 and 16-byte aligned
+// buffers; falls back to the register kernel otherwise.
+int do_gather_tma(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* const* out, int nout, void* ws,
+                  cudaStream_t s);
 
 int do_gather(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* const* out, int nout,
               cudaStream_t s) {
@@ -282,6 +314,35 @@ int do_gather(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* const*
   if (gx < 1) gx = 1;
   zb::gather_layer_kernel<<<dim3(gx, Nd), zb::kThreads, 0, s>>>(a);
   return check_launch("gather_layer_kernel launch");
+}
+
+int do_gather_tma(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* const* out, int nout, void* ws,
+                  cudaStream_t s) {
+  if (L == 0) return ZERO_OK;
+  bool al = true;
+  int rc = check_ptrs(shards, Nd, "shards", &al);
+  if (rc) return rc;
+  rc = check_ptrs(out, nout, "out", &al);
+  if (rc) return rc;
+  const int64_t S = (L + Nd - 1) / Nd;
+  if (!al || S % 8 != 0 || !ws) return do_gather(shards, Nd, L, out, nout, s);
+  int sms = 0;
+  if ((rc = tma_setup(&sms))) return rc;
+  zb::GatherTmaArgs a;
+  std::memset(&a, 0, sizeof a);
+  for (int r = 0; r < Nd; ++r) a.shards[r] = shards[r];
+  for (int o = 0; o < nout; ++o) a.out[o] = out[o];
+  a.Nd = Nd;
+  a.nout = nout;
+  a.L = L;
+  a.S = S;
+  a.hdr = header(ws);
+  const int64_t chunks = (S + zb::kGTile - 1) / zb::kGTile;
+  int64_t gx = ((int64_t)sms * gather_tma_per_sm() + Nd - 1) / Nd;  // about one wave over the Nd rows
+  if (gx > chunks) gx = chunks;
+  if (gx < 1) gx = 1;
+  zb::gather_layer_tma_kernel<<<dim3((unsigned)gx, Nd), 32, zb::kGSmemBytes, s>>>(a);
+  return check_launch("gather_layer_tma_kernel launch");
 }
 
 }  // namespace
@@ -500,6 +561,8 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
     const int64_t L = bucket > 0 ? bucket : N;
     const int64_t nl = (N + L - 1) / L;
+    const bool g16 = (st->flags & ZERO_BF16_GRAD_SHARD) != 0;
+    uint16_t* gsh16 = reinterpret_cast<uint16_t*>(st->grad_shard);
     prof_mark(true, s);
     int64_t off = 0;
     for (int64_t l = 0; l < nl; ++l) {  // forward gathers + backward reduce-scatters, layer by layer
@@ -513,15 +576,20 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
         outs[r] = st->params[r] + l * st->param_layer_stride;
         gl[r] = st->grads[r] + l * st->grad_layer_stride;
       }
-      if ((rc = do_gather(shards, Nd, Ll, outs, Nd, s))) return rc;
+      rc = (st->flags & ZERO_NO_TMA) ? do_gather(shards, Nd, Ll, outs, Nd, s)
+                                     : do_gather_tma(shards, Nd, Ll, outs, Nd, ws, s);
+      if (rc) return rc;
       zb::RsArgs a;
       std::memset(&a, 0, sizeof a);
-      bool ral = aligned16(st->grad_shard + off);
+      bool ral = g16 ? aligned16(gsh16 + off) : aligned16(st->grad_shard + off);
       for (int r = 0; r < Nd; ++r) {
         a.grads[r] = gl[r];
         ral = ral && aligned16(gl[r]);
       }
-      a.out = st->grad_shard + off;
+      if (g16)
+        a.out16 = gsh16 + off;
+      else
+        a.out = st->grad_shard + off;
       a.lo = 0;
       a.hi = Ll;
       a.inv = c.inv;
@@ -543,7 +611,10 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       a.p[0] = a.p[1] = st->master[0] + off;
       a.m[0] = a.m[1] = st->exp_avg[0] + off;
       a.v[0] = a.v[1] = st->exp_avg_sq[0] + off;
-      a.g = st->grad_shard + off;
+      if (g16)
+        a.g16 = gsh16 + off;
+      else
+        a.g = st->grad_shard + off;
       a.out16 = st->param_shard + off;
       a.lo = 0;
       a.hi = Ll;
@@ -551,8 +622,8 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       a.hdr = header(ws);
       a.part = partials(ws);
       a.mode = l == nl - 1 ? zb::kFinalize : 0;
-      a.vec = aligned16(a.p[0]) && aligned16(a.m[0]) && aligned16(a.v[0]) && aligned16(a.g) &&
-              aligned16(a.out16);
+      a.vec = aligned16(a.p[0]) && aligned16(a.m[0]) && aligned16(a.v[0]) &&
+              (g16 ? aligned16(a.g16) : aligned16(a.g)) && aligned16(a.out16);
       if ((rc = launch_adam(a, s))) return rc;
       off += Sl * Nd;
     }
@@ -567,15 +638,22 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   const int64_t B = bucket > 0 ? bucket : N;
   const int64_t nb = (N + B - 1) / B;
 
+  if ((st->flags & ZERO_BF16_GRAD_SHARD) && !(st->flags & ZERO_TWO_PASS))
+    return fail(ZERO_EINVAL, "ZERO_BF16_GRAD_SHARD needs a gradient shard: ZERO_TWO_PASS or stage 3");
   if (st->flags & ZERO_TWO_PASS) {
     if (!st->master[0] || !st->exp_avg[0] || !st->exp_avg_sq[0] || !st->grad_shard)
       return fail(ZERO_EINVAL, "ZERO_TWO_PASS needs master[0], exp_avg[0], exp_avg_sq[0], grad_shard");
+    const bool g16 = (st->flags & ZERO_BF16_GRAD_SHARD) != 0;
+    uint16_t* gsh16 = reinterpret_cast<uint16_t*>(st->grad_shard);
     prof_mark(true, s);
     for (int64_t k = 0; k < nb; ++k) {
       zb::RsArgs a;
       std::memset(&a, 0, sizeof a);
       for (int r = 0; r < Nd; ++r) a.grads[r] = st->grads[r];
-      a.out = st->grad_shard;
+      if (g16)
+        a.out16 = gsh16;
+      else
+        a.out = st->grad_shard;
       a.lo = k * B;
       a.hi = (k + 1) * B < N ? (k + 1) * B : N;
       a.inv = c.inv;
@@ -597,7 +675,10 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
         a.m[i] = two ? st->exp_avg[i] : st->exp_avg[0];
         a.v[i] = two ? st->exp_avg_sq[i] : st->exp_avg_sq[0];
       }
-      a.g = st->grad_shard;
+      if (g16)
+        a.g16 = gsh16;
+      else
+        a.g = st->grad_shard;
       for (int r = 0; r < Nd; ++r) a.reps[r] = st->params[r];
       a.nrep = Nd;
       a.use_live = 1;
@@ -608,7 +689,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       a.part = partials(ws);
       a.mode = k == nb - 1 ? zb::kFinalize : 0;
       a.vec = al && aligned16(a.p[0]) && aligned16(a.p[1]) && aligned16(a.m[0]) && aligned16(a.m[1]) &&
-              aligned16(a.v[0]) && aligned16(a.v[1]) && aligned16(a.g);
+              aligned16(a.v[0]) && aligned16(a.v[1]) && aligned16(st->grad_shard);
       if ((rc = launch_adam(a, s))) return rc;
     }
     prof_mark(false, s);

@@ -432,7 +432,8 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
 
 struct RsArgs {
   const uint16_t* grads[kMaxNd];
-  float* out;        // reduced gradient, indexed like the replicas
+  float* out;        // reduced gradient, indexed like the replicas (fp32 variant)
+  uint16_t* out16;   // reduced gradient rounded to bf16 (bf16 variant)
   int64_t lo, hi;
   float inv;         // static unscale factor
   double inv_base;   // Nd or 1, for the dynamic loss scale
@@ -443,7 +444,11 @@ struct RsArgs {
   int vec;
 };
 
-template <int DT>
+// bf16 round trip of a reduced gradient value (nearest even), as the bf16 variant keeps it.
+__device__ __forceinline__ float round_bf16(float x) { return __uint_as_float((uint32_t)to_bf16(x) << 16); }
+
+// OUT16: keep the reduced gradient as bf16; the flag and the norm then use the rounded value.
+template <int DT, bool OUT16>
 __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_constant__ RsArgs a) {
   __shared__ float s_inv;
   if (threadIdx.x == 0) {
@@ -465,18 +470,27 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       s[k] = __fmul_rn(s[k], inv);
+      if (OUT16) s[k] = round_bf16(s[k]);
       bad |= nonfinite(s[k]);
       sq = __dadd_rn(sq, __dmul_rn((double)s[k], (double)s[k]));
     }
-    st_stream(out + i, make_float4(s[0], s[1], s[2], s[3]));
-    st_stream(out + i + 4, make_float4(s[4], s[5], s[6], s[7]));
+    if (OUT16) {
+      st_stream(a.out16 + i, pack_bf16x8(s));  // exact: the values are already bf16
+    } else {
+      st_stream(out + i, make_float4(s[0], s[1], s[2], s[3]));
+      st_stream(out + i + 4, make_float4(s[4], s[5], s[6], s[7]));
+    }
   }
   for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
     const int64_t i = sp8.scalar_index(a.lo, e);
-    const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), inv);
+    float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), inv);
+    if (OUT16) g = round_bf16(g);
     bad |= nonfinite(g);
     sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
-    out[i] = g;
+    if (OUT16)
+      a.out16[i] = to_bf16(g);
+    else
+      out[i] = g;
   }
   block_finish(sq, bad, a.hdr, a.part, a.mode);
 }
@@ -487,7 +501,8 @@ struct AdamArgs {
   float* p[2];        // state copies; the kernel updates copy `live` in place
   float* m[2];
   float* v[2];
-  const float* g;     // reduced gradient
+  const float* g;     // reduced gradient (fp32 variant)
+  const uint16_t* g16;  // reduced gradient kept as bf16 (bf16 variant)
   uint16_t* out16;    // optional bf16 copy of the new weights (ZeRO-3 shard)
   uint16_t* reps[kMaxNd];  // optional bf16 replicas (fused all-gather of the two-pass path)
   int nrep;
@@ -500,6 +515,7 @@ struct AdamArgs {
   int vec;
 };
 
+template <bool G16>
 __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ AdamArgs a) {
   __shared__ Bias s_bias;
   __shared__ int s_live, s_skip;
@@ -526,7 +542,17 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
       unpack(ld_stream(P_ + i), ld_stream(P_ + i + 4), P);
       unpack(ld_stream(M_ + i), ld_stream(M_ + i + 4), M);
       unpack(ld_stream(V_ + i), ld_stream(V_ + i + 4), V);
-      unpack(ld_stream(G_ + i), ld_stream(G_ + i + 4), G);
+      if (G16) {
+        const uint4 q = ld_stream(a.g16 + i);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          G[2 * k] = __uint_as_float(w[k] << 16);
+          G[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        }
+      } else {
+        unpack(ld_stream(G_ + i), ld_stream(G_ + i + 4), G);
+      }
 #pragma unroll
       for (int k = 0; k < 8; ++k) adam_elem(__fmul_rn(G[k], coef), P[k], M[k], V[k], a.c, b);
       st_stream(P_ + i, make_float4(P[0], P[1], P[2], P[3]));
@@ -544,7 +570,8 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
     for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
       const int64_t i = sp8.scalar_index(a.lo, e);
       float P = P_[i], M = M_[i], V = V_[i];
-      adam_elem(__fmul_rn(G_[i], coef), P, M, V, a.c, b);
+      const float gi = G16 ? __uint_as_float((uint32_t)a.g16[i] << 16) : G_[i];
+      adam_elem(__fmul_rn(gi, coef), P, M, V, a.c, b);
       P_[i] = P;
       M_[i] = M;
       V_[i] = V;

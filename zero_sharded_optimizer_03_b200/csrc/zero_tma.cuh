@@ -377,3 +377,94 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
 }
 
 }  // namespace zb
+
+namespace zb {
+
+// ------------------------------------------------------------------ TMA ZeRO-3 layer gather
+//
+// The gather is a pure fan-out copy: 2 bytes read and 2*nout written per element.  Issued as
+// 16-byte stores from registers it saturates the load/store units (lg_throttle stalls) before
+// DRAM; here one thread per CTA drives the Tensor Memory Accelerator instead: a 1-D bulk load of
+// a chunk of the source shard into shared memory (the next chunk prefetched while the current
+// one is stored), then nout bulk stores of that one shared tile.  A stage is refilled only once
+// the stores that read it have finished reading (bulk async-group accounting).  Waits are
+// bounded as in the fused kernel; a timeout sets the workspace error word.
+
+constexpr int kGTile = 4096;   // elements per chunk (8 KB)
+constexpr int kGStages = 4;
+constexpr size_t kGSmemBytes = (size_t)kGStages * kGTile * 2 + kGStages * sizeof(uint64_t);
+
+struct GatherTmaArgs {
+  const uint16_t* shards[kMaxNd];
+  uint16_t* out[kMaxNd];
+  int Nd, nout;
+  int64_t L, S;
+  Header* hdr;  // error word
+};
+
+__device__ __forceinline__ void bulk_wait_read_2() { asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory"); }
+
+// grid.y = source rank r, grid.x strides over the chunks of shard r; 32 threads per CTA.
+__global__ void __launch_bounds__(32) gather_layer_tma_kernel(const __grid_constant__ GatherTmaArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kGStages * kGTile * 2);
+  const int r = blockIdx.y;
+  const int64_t base = (int64_t)r * a.S;
+  int64_t len = a.L - base;
+  if (len > a.S) len = a.S;
+  if (len <= 0) return;
+  const int64_t len8 = len & ~int64_t(7);  // bulk part (multiples of 16 bytes)
+  const int64_t nchunks = (len8 + kGTile - 1) / kGTile;
+  const int64_t mine = nchunks > (int64_t)blockIdx.x ? (nchunks - 1 - (int64_t)blockIdx.x) / gridDim.x + 1 : 0;
+  const uint16_t* src = a.shards[r];
+  if (threadIdx.x == 0 && mine > 0 && (smem_u32(smem) & 127u) == 0) {
+    for (int k = 0; k < kGStages; ++k) mbar_init(smem_u32(&bars[k]), 1);
+    fence_barrier_init();
+    auto chunk = [&](int64_t it, int64_t* k0, uint32_t* bytes) {
+      *k0 = ((int64_t)blockIdx.x + it * gridDim.x) * kGTile;
+      const int64_t n = len8 - *k0 < kGTile ? len8 - *k0 : kGTile;
+      *bytes = (uint32_t)(n * 2);
+    };
+    auto load = [&](int64_t it) {
+      int64_t k0;
+      uint32_t bytes;
+      chunk(it, &k0, &bytes);
+      const int s = (int)(it % kGStages);
+      mbar_expect_tx(smem_u32(&bars[s]), bytes);
+      bulk_load(smem_u32(smem + (size_t)s * kGTile * 2), src + k0, bytes, smem_u32(&bars[s]));
+    };
+    volatile int abort = 0;
+    int64_t issued = 1;
+    load(0);
+    for (int64_t it = 0; it < mine; ++it) {
+      if (it + 1 < mine) {
+        bulk_wait_read_2();  // the stage chunk it+1 will use was last read by the stores of it-3
+        load(it + 1);
+        issued = it + 2;
+      }
+      const int s = (int)(it % kGStages);
+      if (!wait_bounded(smem_u32(&bars[s]), (uint32_t)((it / kGStages) & 1), &abort)) break;
+      int64_t k0;
+      uint32_t bytes;
+      chunk(it, &k0, &bytes);
+      for (int o = 0; o < a.nout; ++o) bulk_store(a.out[o] + base + k0, smem_u32(smem + (size_t)s * kGTile * 2), bytes);
+      bulk_commit();
+    }
+    bulk_wait_all();
+    if (abort) {
+      atomicOr(&a.hdr->error, kErrTimeout);
+      for (int64_t it = issued > 2 ? issued - 2 : 0; it < issued; ++it)  // loads still in flight
+        wait_drain(smem_u32(&bars[it % kGStages]), (uint32_t)((it / kGStages) & 1));
+    }
+  } else if (threadIdx.x == 0 && mine > 0) {
+    atomicOr(&a.hdr->error, kErrTimeout);  // misaligned shared memory: nothing copied
+  }
+  __syncwarp();
+  if (blockIdx.x == 0)  // the last < 8 elements of the shard
+    for (int64_t k = len8 + threadIdx.x; k < len; k += 32) {
+      const uint16_t w = src[k];
+      for (int o = 0; o < a.nout; ++o) a.out[o][base + k] = w;
+    }
+}
+
+}  // namespace zb
