@@ -300,6 +300,91 @@ def run_offload(args, w, world, rank, dist, dev, config):
         dist.destroy_process_group()
 
 
+# ----------------------------------------------------------------------------- real ranks
+
+def run_dist(args, w, config):
+    """Data parallelism over real GPUs (one process per GPU, torchrun): rank r owns shard r of
+    the workload's N parameters and runs the fused kernel over peer memory (symmetric memory);
+    Nd = the number of GPUs.  Total work is fixed: strong scaling."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import zero_sharded_optimizer_03_b200 as zero
+    from zero_sharded_optimizer_03_b200.dist import DistZero
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29631")
+    os.environ.setdefault("RANK", "0")
+    os.environ.setdefault("WORLD_SIZE", "1")
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    rank, world = dist.get_rank(), dist.get_world_size()
+    N = w["N"]
+    dz = DistZero(N)
+    sp = torch.cuda.current_stream().cuda_stream
+    synth.fill_device(dz.master[0].data_ptr(), synth.NORMAL, synth.F32, synth.SEED,
+                      synth.MASTER_STREAM, dz.hi - dz.lo, 0.02, first=dz.lo, cuda_stream=sp)
+    synth.fill_device(dz.grad.data_ptr(), synth.NORMAL, synth.BF16, synth.SEED,
+                      synth.grad_stream(1, rank), N, w["sigma"], cuda_stream=sp)
+    dz.init(0)
+    dz.publish_weights()
+    hp = zero.hparams(**w["hp"])
+    for _ in range(args.warmup):
+        dz.step(hp)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in kev:
+        a.record()
+        b.record()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for k in range(args.steps):
+        zero.zero_profile_events(kev[k][0].cuda_event, kev[k][1].cuda_event)
+        dz.step(hp)
+    t1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms_total, kern_ms = max_over_ranks(
+        [t0.elapsed_time(t1), sum(a.elapsed_time(b) for a, b in kev) / args.steps], dist, dev)
+    res = dz.result()
+    assert res["overflow"] == 0, res
+    ms = ms_total / args.steps
+    S = dz.S
+    hbm_bytes = S * (2 + 24 + 2)                   # own gradient, state, own replica (per rank)
+    link_bytes = S * 2 * (world - 1) * 2           # peers' gradients in + weights out
+    t_hbm = hbm_bytes / 6527.8e9
+    t_link = link_bytes / 770e9
+    bound = "nvlink" if t_link > t_hbm else "hbm"
+    ideal = max(t_hbm, t_link)
+    if rank == 0:
+        config.update({"Nd": world, "path": "real ranks: fused kernel over peer memory + NCCL "
+                       "step totals", "kernel": "fused_step_kernel (peer loads/stores)",
+                       "parallelism": "dp%d (one rank per GPU)" % world})
+        line = {"metric": METRIC, "value": N / (ms / 1e3), "unit": "params/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic", "config": config,
+                "roofline": {"bound": bound, "achieved": (hbm_bytes if bound == "hbm" else
+                                                          link_bytes) / (kern_ms / 1e3) / 1e9,
+                             "peak": 6527.8 if bound == "hbm" else 770.0, "unit": "GB/s",
+                             "frac": ideal / (kern_ms / 1e3), "traffic": None,
+                             "kernel_ms": kern_ms, "hbm_bytes_per_rank": hbm_bytes,
+                             "nvlink_bytes_per_rank": link_bytes},
+                "cpu_baseline": None, "e2e": None, "clocks": None,
+                "gpu_launches": 3 * args.steps}
+        print(json.dumps(line), flush=True)
+    dz.close()
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -309,6 +394,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--dist", action="store_true",
+                    help="real data parallelism: one rank per GPU owns one shard (Nd = GPUs)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -352,6 +439,9 @@ def main():
               "weights_dtype": "bf16", "parallelism": "replicas (%d simulated ranks per GPU)"
               % w["Nd"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
               % (2 * w["Nd"] * w["N"] / 1e9)}
+
+    if args.dist and args.impl != "reference":
+        return run_dist(args, w, config)
 
     if args.impl == "reference":
         if rank != 0:

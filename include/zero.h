@@ -316,6 +316,30 @@ int zero_reduce_scatter_noalloc(const uint16_t *const *grads, int dtype, int Nd,
  * clears.  Units of a CTA are numbered ceil(Nd/8) gradient chunks then one state unit per tile. */
 int zero_test_inject_stall(int64_t unit);
 
+/* ------------------------------------------------------------------ one GPU per rank */
+
+/* The fused pass of zero_step (ZERO_FUSED) over the window [lo, hi) only, for a data-parallel
+ * rank that owns that window ([P1] §二, [P3] core operations) when the Nd ranks are real GPUs:
+ * st->grads[q] and st->params[q] are then the peer-mapped addresses of rank q's gradient and
+ * weight buffers (e.g. symmetric memory), so the rank-order fan-in reads the peers' gradients over
+ * NVLink and the bf16 results are stored straight into every peer's weight replica -- the
+ * reduce-scatter, the update and the all-gather in one kernel over peer memory.  The fp32
+ * state pointers are the rank's state indexed by global position (base + lo addresses its
+ * first element).  finalize = 0 leaves the step open: the caller combines the pending
+ * overflow flag (MAX) and sum of squares (SUM) of every rank in the workspace header (int32 at
+ * byte 4, double at byte 8), then calls zero_end_step_flip and zero_repair_window; finalize != 0
+ * ends the step here (single GPU).  No clipping (it needs the global norm first).  Async. */
+int zero_fused_window(int Nd, int64_t lo, int64_t hi, const zero_state_t *st,
+                      const zero_hparams_t *hp, int finalize, void *stream);
+
+/* zero_end_step for the fused path: ends the step and, if the combined overflow flag is clear,
+ * makes the state copy written by the fused pass the live one.  Async. */
+int zero_end_step_flip(void *ws, void *stream);
+
+/* After an overflowed (skipped) step, rewrites the window [lo, hi) of every weight replica in
+ * st->params from the unchanged live master weights; does nothing after a clean step.  Async. */
+int zero_repair_window(int Nd, int64_t lo, int64_t hi, const zero_state_t *st, void *stream);
+
 /* ------------------------------------------------------------------ ZeRO-Offload */
 
 /* Buffers of an offloaded step ([P2] "ZeRO-Offload": optimizer state and gradients in CPU

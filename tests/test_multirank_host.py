@@ -53,3 +53,37 @@ def test_reference_arm_other_ranks_exit_without_work():
                           "--gpus", "2", "--steps", "1", "--warmup", "3"], env=env,
                          capture_output=True, text=True, timeout=120)
     assert res.returncode == 0 and res.stdout.strip() == ""
+
+
+def _dist_worker(rank, world, port, out):
+    import datetime
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from zero_sharded_optimizer_03_b200.dist import combine_step_totals, rank_window
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    ws = torch.zeros(16, dtype=torch.uint8)  # the pending totals sit at bytes 4 and 8
+    flag = ws[4:8].view(torch.int32)
+    sumsq = ws[8:16].view(torch.float64)
+    flag.fill_(1 if rank == 1 else 0)
+    sumsq.fill_(0.25 * (rank + 1))
+    combine_step_totals(flag, sumsq)
+    out[rank] = (int(flag.item()), float(sumsq.item()),
+                 [rank_window(1_000_003, world, q) for q in range(world)])
+    dist.destroy_process_group()
+
+
+def test_dist_step_totals_and_windows_two_gloo_ranks():
+    world, port = 2, 29623
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_dist_worker, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 1          # any rank's overflow skips every rank
+    assert res[0][1] == res[1][1] == 0.75       # sums of squares add up
+    windows = res[0][2]
+    assert windows == [(0, 500002, 500002), (500002, 1000003, 500002)]

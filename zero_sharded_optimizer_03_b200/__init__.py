@@ -19,6 +19,7 @@ __all__ = [
     "zero_allgather", "zero_end_step", "zero3_gather_layer", "zero_step",
     "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events",
     "zero_test_inject_stall", "zero_loss_scaler_init", "zero_host_adam", "zero_offload_step",
+    "zero_fused_window", "zero_end_step_flip", "zero_repair_window",
     "ZeroOffloadBuffers",
     "zero_reduce_scatter_noalloc", "ZERO_NOALLOC_MAX_WINDOW", "hparams", "ZeroBuffers",
     "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_NO_TMA",
@@ -117,6 +118,11 @@ def _load() -> ctypes.CDLL:
         "zero_profile_events": ([_P, _P], ctypes.c_int),
         "zero_test_inject_stall": ([_i64], ctypes.c_int),
         "zero_loss_scaler_init": ([_P, _dbl, _dbl, _dbl, _i64, _P], ctypes.c_int),
+        "zero_fused_window": ([ctypes.c_int, _i64, _i64, ctypes.POINTER(zero_state_t),
+                               ctypes.POINTER(zero_hparams_t), ctypes.c_int, _P], ctypes.c_int),
+        "zero_end_step_flip": ([_P, _P], ctypes.c_int),
+        "zero_repair_window": ([ctypes.c_int, _i64, _i64, ctypes.POINTER(zero_state_t), _P],
+                               ctypes.c_int),
         "zero_host_adam": ([_P, _P, _P, _P, _i64, ctypes.POINTER(zero_hparams_t), _i64,
                             ctypes.c_float, _P, ctypes.c_int], ctypes.c_int),
         "zero_offload_step": ([ctypes.c_int, _i64, _i64, ctypes.POINTER(zero_offload_state_t),
@@ -214,6 +220,20 @@ def zero_reduce_scatter_noalloc(grads, dtype: int, Nd: int, lo: int, hi: int,
     zero_rs_summary_t (16 bytes) that receives the window's overflow flag and sum of squares."""
     _check(lib.zero_reduce_scatter_noalloc(_ptrs(grads), dtype, Nd, lo, hi, ctypes.byref(hp),
                                            grad_out, summary, 1 if accumulate else 0, stream))
+
+
+def zero_fused_window(Nd: int, lo: int, hi: int, state: zero_state_t, hp: zero_hparams_t,
+                      finalize: bool = False, stream: int = 0) -> None:
+    _check(lib.zero_fused_window(Nd, lo, hi, ctypes.byref(state), ctypes.byref(hp),
+                                 1 if finalize else 0, stream))
+
+
+def zero_end_step_flip(ws: int, stream: int = 0) -> None:
+    _check(lib.zero_end_step_flip(ws, stream))
+
+
+def zero_repair_window(Nd: int, lo: int, hi: int, state: zero_state_t, stream: int = 0) -> None:
+    _check(lib.zero_repair_window(Nd, lo, hi, ctypes.byref(state), stream))
 
 
 def zero_host_adam(master: int, exp_avg: int, exp_avg_sq: int, grad: int, n: int,

@@ -1061,3 +1061,73 @@ extern "C" int zero_offload_step(int Nd, int64_t N, int64_t chunk, const zero_of
   // the events may be destroyed now: pending work that refers to them still completes
   return ZERO_OK;
 }
+
+// ==================================================================== windows (multi-GPU)
+
+extern "C" int zero_fused_window(int Nd, int64_t lo, int64_t hi, const zero_state_t* st, const zero_hparams_t* hp,
+                                 int finalize, void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if ((rc = check_window(lo, hi))) return rc;
+  if ((rc = check_hp(hp))) return rc;
+  if (!st || !st->workspace) return fail(ZERO_EINVAL, "state or workspace is NULL");
+  if (st->grad_dtype != ZERO_BF16 && st->grad_dtype != ZERO_FP16) return fail(ZERO_EINVAL, "grad_dtype=%d", st->grad_dtype);
+  if (hp->max_grad_norm > 0) return fail(ZERO_EINVAL, "the fused pass cannot clip (needs the global norm first)");
+  bool al = true;
+  if ((rc = check_ptrs(st->grads, Nd, "grads", &al))) return rc;
+  if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
+  zb::FusedArgs a;
+  std::memset(&a, 0, sizeof a);
+  for (int r = 0; r < Nd; ++r) {
+    a.grads[r] = st->grads[r];
+    a.reps[r] = st->params[r];
+  }
+  for (int i = 0; i < 2; ++i) {
+    if (!st->master[i] || !st->exp_avg[i] || !st->exp_avg_sq[i])
+      return fail(ZERO_EINVAL, "the fused pass needs both state copies");
+    a.p[i] = st->master[i];
+    a.m[i] = st->exp_avg[i];
+    a.v[i] = st->exp_avg_sq[i];
+    al = al && aligned16(a.p[i]) && aligned16(a.m[i]) && aligned16(a.v[i]);
+  }
+  a.c = make_consts(hp, Nd);
+  a.hdr = header(st->workspace);
+  a.part = partials(st->workspace);
+  a.Nd = Nd;
+  a.vec = al;
+  a.lo = lo;
+  a.hi = hi;
+  a.mode = zb::kAccSet | (finalize ? (zb::kFinalize | zb::kFlip) : 0);
+  cudaStream_t s = (cudaStream_t)stream;
+  prof_mark(true, s);
+  rc = launch_fused(st->grad_dtype, a, s);
+  prof_mark(false, s);
+  return rc;
+}
+
+extern "C" int zero_end_step_flip(void* ws, void* stream) {
+  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  return launch_ws(ws, zb::kWsEndFlip, 0, (cudaStream_t)stream);
+}
+
+extern "C" int zero_repair_window(int Nd, int64_t lo, int64_t hi, const zero_state_t* st, void* stream) {
+  int rc = check_nd(Nd);
+  if (rc) return rc;
+  if ((rc = check_window(lo, hi))) return rc;
+  if (!st || !st->workspace || !st->master[0] || !st->master[1]) return fail(ZERO_EINVAL, "state is incomplete");
+  if (lo == hi) return ZERO_OK;
+  bool al = aligned16(st->master[0]) && aligned16(st->master[1]);
+  if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
+  zb::CastArgs r;
+  std::memset(&r, 0, sizeof r);
+  r.src[0] = st->master[0];
+  r.src[1] = st->master[1];
+  for (int q = 0; q < Nd; ++q) r.reps[q] = st->params[q];
+  r.nrep = Nd;
+  r.gate = zb::kGateRepair;
+  r.lo = lo;
+  r.hi = hi;
+  r.hdr = header(st->workspace);
+  r.vec = al;
+  return launch_cast(r, (cudaStream_t)stream);
+}

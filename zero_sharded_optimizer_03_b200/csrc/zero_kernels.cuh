@@ -675,7 +675,7 @@ __global__ void __launch_bounds__(kThreads) gather_layer_kernel(const __grid_con
 
 // ------------------------------------------------------------------ workspace control
 
-enum : int { kWsInit = 0, kWsBegin = 1, kWsEnd = 2 };
+enum : int { kWsInit = 0, kWsBegin = 1, kWsEnd = 2, kWsEndFlip = 3 };
 
 __global__ void ws_ctl_kernel(Header* h, int op, long long t0) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
@@ -698,7 +698,7 @@ __global__ void ws_ctl_kernel(Header* h, int op, long long t0) {
     h->pending_flag = 0;
     h->pending_sumsq = 0.0;
   }
-  if (op == kWsEnd) end_step(h, 0);
+  if (op == kWsEnd || op == kWsEndFlip) end_step(h, op == kWsEndFlip);
   __threadfence();
 }
 
