@@ -12,12 +12,12 @@ import zero_sharded_optimizer_03_b200 as zero
 
 SEED = synth.SEED
 
-# Hyperparameters of the workloads (readings: torch AdamW defaults where unstated).
-HP_C1 = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, loss_scale=1.0)
-HP_C2 = dict(lr=6e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)
-HP_C3 = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1024.0)
-HP_C4 = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)
-HP_C5 = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)
+# Hyperparameters of the workloads (torch AdamW defaults where a workload states none).
+HP_ADAM_LR1E3 = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, loss_scale=1.0)
+HP_ADAMW_GPT2 = dict(lr=6e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)
+HP_ADAMW_FP16_LS1024 = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1024.0)
+HP_ADAMW_ZERO3 = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)
+HP_ADAMW_WIDE = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)
 
 LLAMA7B_LAYER = 4 * 4096 * 4096 + 3 * 4096 * 11008  # q,k,v,o + gate,up,down = 202,375,168
 

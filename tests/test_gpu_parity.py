@@ -15,7 +15,7 @@ import torch
 import oracle
 import synth
 import zero_sharded_optimizer_03_b200 as zero
-from _gpu import (HP_C1, HP_C2, HP_C3, HP_C4, HP_C5, LLAMA7B_LAYER, SEED, SampledOracle, at,
+from _gpu import (HP_ADAM_LR1E3, HP_ADAMW_GPT2, HP_ADAMW_FP16_LS1024, HP_ADAMW_ZERO3, HP_ADAMW_WIDE, LLAMA7B_LAYER, SEED, SampledOracle, at,
                   assert_bf16_close, assert_f32_close, boundaries, f32, fill, free, grads_at,
                   put_bits, sample_indices, stream, u16)
 
@@ -77,7 +77,7 @@ def test_device_generator_matches_host(kind, dtype):
 
 @pytest.mark.parametrize("flags", [zero.ZERO_FUSED, zero.ZERO_TWO_PASS])
 @pytest.mark.parametrize("stage", [1, 2])
-def test_config1_zero2_single_step_full(stage, flags):
+def test_zero2_1m_nd4_single_step_full(stage, flags):
     """N = 1,000,003 (padded to ceil(N/4)), Nd = 4, bf16 grads ~N(0,1e-3) per rank, master
     ~N(0,0.02), m = v = 0, Adam lr 1e-3 (wd 0), step 1: every element compared."""
     Nd, N = 4, 1_000_003
@@ -90,10 +90,10 @@ def test_config1_zero2_single_step_full(stage, flags):
                              sigma=1e-3) for r in range(Nd)]
     for r in range(Nd):
         fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(1, r), sigma=1e-3)
-    buf.step(zero.hparams(**HP_C1))
+    buf.step(zero.hparams(**HP_ADAM_LR1E3))
     oreps = [np.zeros(N, np.uint16) for _ in range(Nd)]
-    t, ovf, ss = oracle.zero12_step(Nd, N, 0, oracle.BF16, grads, om, mm, vm, oreps, HP_C1, 0)
-    res = _compare_full(buf, om, mm, vm, oreps, t, ss, "c1")
+    t, ovf, ss = oracle.zero12_step(Nd, N, 0, oracle.BF16, grads, om, mm, vm, oreps, HP_ADAM_LR1E3, 0)
+    res = _compare_full(buf, om, mm, vm, oreps, t, ss, "1M Nd=4")
     assert res["overflow"] == 0 and res["skipped"] == 0
     live = buf.live()
     # every rank's shard view holds exactly that rank's elements; the padding stays zero
@@ -122,7 +122,7 @@ CASES = [(0, 4), (1, 1), (1, 4), (7, 3), (8, 8), (9, 2), (15, 64), (17, 5), (100
                                           (zero.ZERO_TWO_PASS, 0), (zero.ZERO_TWO_PASS, 777)])
 def test_small_ragged_three_steps(N, Nd, gdt, flags, bucket):
     odt, sdt = DT[gdt]
-    hp = dict(HP_C3) if gdt == zero.ZERO_FP16 else dict(HP_C2)
+    hp = dict(HP_ADAMW_FP16_LS1024) if gdt == zero.ZERO_FP16 else dict(HP_ADAMW_GPT2)
     sigma = 1e-4 * 1024 if gdt == zero.ZERO_FP16 else 1e-3
     buf = zero.ZeroBuffers(2, Nd, N, grad_dtype=gdt, flags=flags)
     _init_state(buf, N)
@@ -148,7 +148,7 @@ def test_unaligned_views_take_the_scalar_path():
     """Buffers that start 2 or 4 bytes past a 16-byte boundary are legal and give the same
     results as aligned ones."""
     Nd, N = 3, 5003
-    hp = dict(HP_C2)
+    hp = dict(HP_ADAMW_GPT2)
     S, Np, _ = oracle.partition(N, Nd)
     big = [torch.zeros(N + 1, dtype=torch.bfloat16, device="cuda") for _ in range(2 * Nd)]
     st_big = [torch.zeros(Np + 1, dtype=torch.float32, device="cuda") for _ in range(6)]
@@ -202,7 +202,7 @@ def test_tma_and_register_kernels_identical(Nd, gdt):
         for k in (1, 2):
             for r in range(Nd):
                 fill(buf.grads[r], synth.NORMAL, sdt, synth.grad_stream(k, r), sigma=1e-3)
-            buf.step(zero.hparams(**HP_C2), bucket=100_001)
+            buf.step(zero.hparams(**HP_ADAMW_GPT2), bucket=100_001)
         res = buf.result()
         live = buf.live()
         outs.append((res, f32(buf.master[live]).tobytes(), f32(buf.exp_avg[live]).tobytes(),
@@ -225,7 +225,7 @@ def test_stage1_and_stage2_identical():
         for k in (1, 2):
             for r in range(Nd):
                 fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(k, r), sigma=1e-3)
-            buf.step(zero.hparams(**HP_C2))
+            buf.step(zero.hparams(**HP_ADAMW_GPT2))
         live = buf.live()
         outs.append((f32(buf.master[live]).tobytes(), u16(buf.params[5]).tobytes()))
         del buf
@@ -241,7 +241,7 @@ def test_bucketed_equals_unbucketed_and_repeatable():
         _init_state(buf, N)
         for r in range(Nd):
             fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(1, r), sigma=1e-3)
-        buf.step(zero.hparams(**HP_C2), bucket=bucket)
+        buf.step(zero.hparams(**HP_ADAMW_GPT2), bucket=bucket)
         live = buf.live()
         outs.append((f32(buf.master[live]).tobytes(), f32(buf.exp_avg_sq[live]).tobytes(),
                      u16(buf.params[3]).tobytes()))
@@ -256,7 +256,7 @@ def test_bucketed_equals_unbucketed_and_repeatable():
 @pytest.mark.parametrize("bad", [0x7F80, 0xFF80, 0x7FC1, "pair"])
 def test_overflow_skips_then_recovers(flags, bad):
     Nd, N = 4, 200_003
-    hp = dict(HP_C2)
+    hp = dict(HP_ADAMW_GPT2)
     buf = zero.ZeroBuffers(2, Nd, N, flags=flags)
     _init_state(buf, N, t0=10)
     S, Np, _ = oracle.partition(N, Nd)
@@ -312,7 +312,7 @@ def test_bounded_wait_gives_up_reports_error_and_device_stays_usable():
     the GPU: the consumers give up after 1 s, the step is skipped with the error word set, the
     state and replicas keep their values, and the next step runs normally."""
     Nd, N = 8, 2048 * 400
-    hp = dict(HP_C2)
+    hp = dict(HP_ADAMW_GPT2)
     buf = zero.ZeroBuffers(2, Nd, N, flags=zero.ZERO_FUSED | zero.ZERO_FORCE_TMA)
     _init_state(buf, N)
     for r in range(Nd):
@@ -531,7 +531,7 @@ def test_offload_step_matches_oracle(gdt, dynamic, max_norm):
 def test_building_blocks_two_pass_matches_oracle():
     """begin -> reduce_scatter (per rank's shard) -> adam (per shard) -> allgather -> end."""
     Nd, N = 5, 123_457
-    hp = dict(HP_C3)
+    hp = dict(HP_ADAMW_FP16_LS1024)
     S, Np, _ = oracle.partition(N, Nd)
     sigma = 0.1024
     grads = [torch.zeros(N, dtype=torch.float16, device="cuda") for _ in range(Nd)]
@@ -582,7 +582,7 @@ def test_building_blocks_two_pass_matches_oracle():
 def test_empty_step_advances_t():
     buf = zero.ZeroBuffers(2, 4, 0)
     buf.init_workspace(5)
-    buf.step(zero.hparams(**HP_C1))
+    buf.step(zero.hparams(**HP_ADAM_LR1E3))
     res = buf.result()
     assert res["step"] == 6 and res["overflow"] == 0 and res["grad_sumsq"] == 0.0
 
@@ -611,7 +611,7 @@ def test_zero3_step_matches_oracle(layer_len, N, Nd):
     then Adam on every shard and the bf16 shard update; three steps, every element."""
     buf = zero.ZeroBuffers(3, Nd, N, layer_len=layer_len, per_layer_buffers=True)
     sizes = buf.layer_sizes
-    hp = dict(HP_C4)
+    hp = dict(HP_ADAMW_ZERO3)
     total = buf.Np
     om = np.zeros(total, np.float32)
     off = 0
@@ -701,12 +701,12 @@ def _sampled_run(stage, Nd, N, steps, hp, gdt, sigma, bucket=0, flags=zero.ZERO_
     return buf, res, so
 
 
-def test_config2_zero1_gpt2_small_ten_steps():
+def test_zero1_gpt2_small_124m_nd8_ten_steps():
     """N = 124,439,808 (GPT-2 small), Nd = 8, ZeRO-1, 10 AdamW steps (lr 6e-4, wd 0.01), fresh
     bf16 grads ~N(0,1e-3) every step, bf16 weights all-gathered to 8 replicas each step."""
     N, Nd = 124_439_808, 8
     S = oracle.partition(N, Nd)[0]
-    buf, res, so = _sampled_run(1, Nd, N, 10, HP_C2, zero.ZERO_BF16, 1e-3,
+    buf, res, so = _sampled_run(1, Nd, N, 10, HP_ADAMW_GPT2, zero.ZERO_BF16, 1e-3,
                                 extra=boundaries(S, N))
     # property at full size: the reduced gradient is the mean of 8 N(0, 1e-3) replicas, so
     # E[sum g^2] = N * 1e-6 / 8 (the generator's variance is 1 - 2^-32)
@@ -716,14 +716,14 @@ def test_config2_zero1_gpt2_small_ten_steps():
     free()
 
 
-def test_config3_zero2_bucketed_fp16_with_overflow():
+def test_zero2_1p3b_nd16_fp16_buckets_with_overflow():
     """N = 1.3e9 in 25M-element buckets, Nd = 16, fp16 grads ~N(0,1e-4)*1024 carrying loss
     scale 1024 (unscaled in the kernel); +inf planted at a seeded (rank, index) on step 3,
     which must skip that step; 5 AdamW steps."""
     N, Nd, B = 1_300_000_000, 16, 25_000_000
     S = oracle.partition(N, Nd)[0]
     site = synth.inject_site(SEED, Nd, N)
-    buf, res, so = _sampled_run(2, Nd, N, 5, HP_C3, zero.ZERO_FP16, 1e-4 * 1024, bucket=B,
+    buf, res, so = _sampled_run(2, Nd, N, 5, HP_ADAMW_FP16_LS1024, zero.ZERO_FP16, 1e-4 * 1024, bucket=B,
                                 inject=(3, site), n_random=50_000,
                                 extra=boundaries(S, N) + boundaries(B, N))
     assert res["step"] == 4 and res["skipped"] == 1
@@ -731,12 +731,12 @@ def test_config3_zero2_bucketed_fp16_with_overflow():
     free()
 
 
-def test_config5_wide_fan_in():
+def test_zero2_2p28_nd64_wide_fan_in():
     """N = 2^28, Nd = 64, bf16 grads ~N(0,1e-3) with 1% of values x1e3 (hash-selected), AdamW
     step 1000 with m ~ |N(0,1e-3)|, v = N(0,1e-6)^2."""
     N, Nd = 1 << 28, 64
     tail = float(np.float32(1e-3 * 1e3))
-    buf, res, so = _sampled_run(2, Nd, N, 1, HP_C5, zero.ZERO_BF16, 1e-3, kind=synth.HEAVY,
+    buf, res, so = _sampled_run(2, Nd, N, 1, HP_ADAMW_WIDE, zero.ZERO_BF16, 1e-3, kind=synth.HEAVY,
                                 tail_sigma=tail, t0=999, m_kind=synth.ABS, v_kind=synth.SQUARE,
                                 m_sigma=1e-3, v_sigma=1e-6, n_random=50_000,
                                 extra=boundaries(N // Nd, N))
@@ -748,15 +748,15 @@ def test_config5_wide_fan_in():
     free()
 
 
-def test_target_2p28_nd8_fused():
+def test_zero2_2p28_nd8_fused():
     N, Nd = 1 << 28, 8
-    buf, res, so = _sampled_run(2, Nd, N, 2, HP_C5, zero.ZERO_BF16, 1e-3, n_random=50_000,
+    buf, res, so = _sampled_run(2, Nd, N, 2, HP_ADAMW_WIDE, zero.ZERO_BF16, 1e-3, n_random=50_000,
                                 extra=boundaries(N // Nd, N))
     del buf
     free()
 
 
-def test_config4_zero3_llama7b_shaped():
+def test_zero3_llama7b_shaped_32_layers_nd8():
     """32 layers of q,k,v,o (4096x4096) + gate,up,down (4096x11008), bf16, Nd = 8; per layer:
     gather the full layer from 8 shards, reduce-scatter 8 bf16 grad replicas ~N(0,1e-3) into
     the fp32 gradient shard; then AdamW on the fp32 shards; 1 step.  Driven through the
@@ -764,7 +764,7 @@ def test_config4_zero3_llama7b_shaped():
     Nd, L, nl = 8, LLAMA7B_LAYER, 32
     N = L * nl
     S = oracle.partition(L, Nd)[0]
-    hp = dict(HP_C4)
+    hp = dict(HP_ADAMW_ZERO3)
     chp = zero.hparams(**hp)
     dev = "cuda"
     master = torch.zeros(N, device=dev)
