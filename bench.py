@@ -193,12 +193,12 @@ def cpu_baseline(w, target_s=10.0, steps=None):
         bucket = min(w.get("bucket", 0), n)
         return oracle.zero12_step(Nd, n, bucket, odt, g, p, m, v, reps, w["hp"], t)[0]
 
-    n0 = 1 << 18
+    n0 = 1 << 16
     g, p, m, v, reps = make(n0)
     t = time.perf_counter()
     one_step(n0, g, p, m, v, reps, 0)
     rate0 = n0 / (time.perf_counter() - t)
-    n = int(min(w["N"], max(n0, rate0 * target_s)))
+    n = int(min(w["N"], max(1 << 12, rate0 * target_s)))
     if w["stage"] == 3:
         n -= n % Nd  # one unpadded layer
     g, p, m, v, reps = make(n)
@@ -411,6 +411,8 @@ def main():
                     help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather")
     ap.add_argument("--bucket-override", type=int, default=-1,
                     help="stages 1/2: run with a different bucket size (0 = one bucket)")
+    ap.add_argument("--nd-override", type=int, default=0,
+                    help="run the workload with a different number of simulated ranks")
     ap.add_argument("--layer-override", type=int, default=0,
                     help="stage 3: run with a different layer length")
     ap.add_argument("--n-override", type=int, default=0,
@@ -421,6 +423,9 @@ def main():
     if args.n_override:
         w["N"] = args.n_override
         w["desc"] += " [N overridden to %d]" % args.n_override
+    if args.nd_override:
+        w["Nd"] = args.nd_override
+        w["desc"] += " [Nd overridden to %d]" % args.nd_override
     if args.layer_override and w["stage"] == 3:
         w["layer"] = w["bucket"] = args.layer_override
         w["desc"] += " [layer overridden to %d]" % args.layer_override
@@ -446,7 +451,10 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        n, times = cpu_baseline(w, target_s=3.0, steps=args.warmup + args.steps)
+        # each step is a bounded sample of the workload, sized so that the whole run of
+        # warmup + steps oracle steps takes about two minutes (at most 3 s per step)
+        per_step = min(3.0, 120.0 / (args.warmup + args.steps))
+        n, times = cpu_baseline(w, target_s=per_step, steps=args.warmup + args.steps)
         timed = times[args.warmup:]
         ms = 1e3 * sum(timed) / len(timed)
         val = n / (ms / 1e3)

@@ -478,6 +478,53 @@ def test_bf16_grad_shard_zero3_and_two_pass_match_oracle(max_norm):
     free()
 
 
+# ----------------------------------------------------------------------------- CUDA graphs
+
+@pytest.mark.parametrize("stage,flags", [(2, zero.ZERO_FUSED), (2, zero.ZERO_FUSED | zero.ZERO_FORCE_TMA),
+                                         (2, zero.ZERO_TWO_PASS), (3, zero.ZERO_FUSED)])
+def test_step_captured_in_a_cuda_graph_matches_eager(stage, flags):
+    """The whole step is device-resident (step counter, live copy, overflow decision and loss
+    scale live in the workspace), so it can be captured once and replayed: three replays with
+    fresh gradients give the same bytes as three eager steps, including a skipped one."""
+    Nd, N, L = 4, 2048 * 40 + 8, 2048 * 10 + 2
+    hp = zero.hparams(lr=1e-3, weight_decay=0.01)
+    outs = []
+    for use_graph in (False, True):
+        buf = (zero.ZeroBuffers(3, Nd, N, layer_len=L, per_layer_buffers=True) if stage == 3
+               else zero.ZeroBuffers(stage, Nd, N, flags=flags))
+        fill(buf.master[0], synth.NORMAL, synth.F32, synth.MASTER_STREAM, n=N, sigma=0.02)
+        buf.init_workspace(0)
+        buf.sync_params_from_master()
+        graph = None
+        side = torch.cuda.Stream()
+        for k in (1, 2, 3):
+            for r in range(Nd):
+                fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(k, r), sigma=1e-3)
+            if k == 2:
+                put_bits(buf.grads[1], 5, 0x7F80)
+            if not use_graph:
+                buf.step(hp)
+                continue
+            if graph is None:
+                side.wait_stream(torch.cuda.current_stream())
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=side):
+                    zero.zero_step(buf.stage, Nd, N, buf.layer_len if stage == 3 else 0, buf.state,
+                                   hp, side.cuda_stream)
+                torch.cuda.current_stream().wait_stream(side)
+            graph.replay()  # capture does not run the work: every step comes from a replay
+        torch.cuda.synchronize()
+        res = buf.result()
+        live = buf.live()
+        outs.append((res["step"], res["skipped"], f32(buf.master[live]).tobytes(),
+                     f32(buf.exp_avg_sq[live]).tobytes(),
+                     u16(buf.param_shard if stage == 3 else buf.params[Nd - 1]).tobytes()))
+        del graph, buf
+    assert outs[0][:2] == outs[1][:2] == (2, 1)
+    assert outs[0] == outs[1]
+    free()
+
+
 # ----------------------------------------------------------------------------- ZeRO-Offload
 
 @pytest.mark.parametrize("gdt,dynamic,max_norm", [(zero.ZERO_BF16, False, 0.0),
