@@ -478,6 +478,62 @@ def test_bf16_grad_shard_zero3_and_two_pass_match_oracle(max_norm):
     free()
 
 
+# ----------------------------------------------------------------------------- randomized
+
+def _random_cases(n_cases=40, seed=2026):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for k in range(n_cases):
+        N = int(rng.choice([0, 1, 7, 9, 63, 4095, 4097, 20_000, 65_536 + 5, 150_001, 300_000]))
+        Nd = int(rng.choice([1, 2, 3, 4, 5, 8, 13, 16, 31, 64]))
+        gdt = int(rng.choice([zero.ZERO_BF16, zero.ZERO_FP16]))
+        path = str(rng.choice(["fused", "tma", "two-pass", "two-pass-g16"]))
+        bucket = int(rng.choice([0, 0, 1000, 2048 * 3 + 5, 50_001]))
+        clip = path.startswith("two-pass") and bool(rng.random() < 0.5)
+        dyn = bool(rng.random() < 0.3)
+        cases.append((k, N, Nd, gdt, path, bucket, clip, dyn))
+    return cases
+
+
+@pytest.mark.parametrize("case", _random_cases(), ids=lambda c: "case%d" % c[0])
+def test_randomized_against_oracle(case):
+    """Seeded random shapes, paths and options, two steps each, every element compared."""
+    k, N, Nd, gdt, path, bucket, clip, dyn = case
+    odt, sdt = DT[gdt]
+    flags = {"fused": zero.ZERO_FUSED, "tma": zero.ZERO_FUSED | zero.ZERO_FORCE_TMA,
+             "two-pass": zero.ZERO_TWO_PASS,
+             "two-pass-g16": zero.ZERO_TWO_PASS | zero.ZERO_BF16_GRAD_SHARD}[path]
+    max_norm = 1e-3 if clip else 0.0
+    ls = 64.0 if gdt == zero.ZERO_FP16 else 1.0
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=ls, max_grad_norm=max_norm,
+              bf16_grad=path == "two-pass-g16", dynamic_scale=dyn, scale_interval=1)
+    buf = zero.ZeroBuffers(2, Nd, N, grad_dtype=gdt, flags=flags)
+    _init_state(buf, N, t0=int(k))
+    if dyn:
+        zero.zero_loss_scaler_init(buf.ws.data_ptr(), ls, 2.0, 0.5, 1, stream())
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    oreps = [oracle.f32_to_bf16(om[:N]) for _ in range(Nd)]
+    t, scale, good = int(k), ls, 0
+    for step in (1, 2):
+        sigma = float(np.float32(1e-3 * scale)) if gdt == zero.ZERO_FP16 else 1e-3
+        hg = [synth.fill_host(synth.NORMAL, sdt, SEED, synth.grad_stream(step, r), N, sigma=sigma)
+              for r in range(Nd)]
+        for r in range(Nd):
+            if N:
+                fill(buf.grads[r], synth.NORMAL, sdt, synth.grad_stream(step, r), n=N,
+                     sigma=sigma)
+        buf.step(zero.hparams(lr=1e-3, weight_decay=0.01, loss_scale=ls,
+                              max_grad_norm=max_norm), bucket=bucket)
+        t, ovf, ss, scale, good = oracle.zero12_step_ex(Nd, N, bucket, odt, hg, om, mm, vm, oreps,
+                                                        hp, t, scale, good)
+    res = _compare_full(buf, om, mm, vm, oreps, t, ss, "case %d" % k)
+    if dyn:
+        assert res["loss_scale"] == scale
+    del buf
+    free()
+
+
 # ----------------------------------------------------------------------------- CUDA graphs
 
 @pytest.mark.parametrize("stage,flags", [(2, zero.ZERO_FUSED), (2, zero.ZERO_FUSED | zero.ZERO_FORCE_TMA),
