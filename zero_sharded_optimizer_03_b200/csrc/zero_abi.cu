@@ -37,14 +37,20 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Resident CTAs per SM for each kernel, cached per device (occupancy does not change).
 constexpr int kMaxDevices = 64;
 enum KernelId {
-  kFusedBf16, kFusedFp16, kRsBf16, kRsFp16, kRsBf16Out16, kRsFp16Out16, kAdam, kAdamG16, kCast, kGather,
+  kFusedBf16, kFusedFp16, kFusedBf16C1, kFusedFp16C1, kFusedBf16C2, kFusedFp16C2, kFusedBf16C4, kFusedFp16C4, kRsBf16, kRsFp16, kRsBf16Out16, kRsFp16Out16, kAdam, kAdamG16, kCast, kGather,
   kNumKernels
 };
 
 const void* kernel_ptr(int id) {
   switch (id) {
-    case kFusedBf16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0>);
-    case kFusedFp16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1>);
+    case kFusedBf16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 8>);
+    case kFusedFp16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 8>);
+    case kFusedBf16C1: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 1>);
+    case kFusedFp16C1: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 1>);
+    case kFusedBf16C2: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 2>);
+    case kFusedFp16C2: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 2>);
+    case kFusedBf16C4: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 4>);
+    case kFusedFp16C4: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 4>);
     case kRsBf16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0, false>);
     case kRsFp16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<1, false>);
     case kRsBf16Out16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0, true>);
@@ -210,16 +216,22 @@ void prof_mark(bool start, cudaStream_t s) {
 
 // ------------------------------------------------------------------ launchers
 
-int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s) {
-  const int kid = dtype == ZERO_FP16 ? kFusedFp16 : kFusedBf16;
+template <int DT, int CH>
+int launch_fused_ch(int kid, const zb::FusedArgs& a, cudaStream_t s) {
   int grid = 0;
   int rc = grid_for(kid, (a.hi - a.lo + 7) / 8, &grid);
   if (rc) return rc;
-  if (dtype == ZERO_FP16)
-    zb::fused_step_kernel<1><<<grid, zb::kThreads, 0, s>>>(a);
-  else
-    zb::fused_step_kernel<0><<<grid, zb::kThreads, 0, s>>>(a);
+  zb::fused_step_kernel<DT, CH><<<grid, zb::kThreads, 0, s>>>(a);
   return check_launch("fused_step_kernel launch");
+}
+
+// The rank batch width follows the fan-in: 1, 2, 4 replicas per batch for Nd <= 4, else 8.
+int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s) {
+  const bool f16 = dtype == ZERO_FP16;
+  if (a.Nd <= 1) return f16 ? launch_fused_ch<1, 1>(kFusedFp16C1, a, s) : launch_fused_ch<0, 1>(kFusedBf16C1, a, s);
+  if (a.Nd <= 2) return f16 ? launch_fused_ch<1, 2>(kFusedFp16C2, a, s) : launch_fused_ch<0, 2>(kFusedBf16C2, a, s);
+  if (a.Nd <= 4) return f16 ? launch_fused_ch<1, 4>(kFusedFp16C4, a, s) : launch_fused_ch<0, 4>(kFusedBf16C4, a, s);
+  return f16 ? launch_fused_ch<1, 8>(kFusedFp16, a, s) : launch_fused_ch<0, 8>(kFusedBf16, a, s);
 }
 
 // TMA-pipelined fused step over [a.lo, a.hi): whole tiles through the bulk-copy pipeline, the

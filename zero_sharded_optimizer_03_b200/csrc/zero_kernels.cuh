@@ -208,18 +208,19 @@ __device__ __forceinline__ void add8(float (&s)[8], const uint4& q) {
 }
 
 // Rank-order sum of the Nd replicas at 8 consecutive elements starting at i (16-byte aligned).
-// Loads are issued 8 ranks at a time so that up to 128 bytes per thread are in flight.
-template <int DT>
+// Loads are issued CH ranks at a time so that up to CH x 16 bytes per thread are in flight; a
+// small CH (small fan-in) leaves registers for more resident warps.
+template <int DT, int CH = 8>
 __device__ __forceinline__ void fan_in8(const uint16_t* const* grads, int Nd, int64_t i, float (&s)[8]) {
 #pragma unroll
   for (int k = 0; k < 8; ++k) s[k] = 0.0f;
-  for (int r0 = 0; r0 < Nd; r0 += 8) {
-    uint4 q[8];
+  for (int r0 = 0; r0 < Nd; r0 += CH) {
+    uint4 q[CH];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < CH; ++u)
       if (r0 + u < Nd) q[u] = ld_stream(grads[r0 + u] + i);
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < CH; ++u)
       if (r0 + u < Nd) add8<DT>(s, q[u]);
   }
 }
@@ -364,8 +365,11 @@ struct FusedArgs {
   int unused;
 };
 
-template <int DT>
-__global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_constant__ FusedArgs a) {
+// CH: gradient replicas loaded per batch (1, 2, 4 or 8).  Built for 3 resident CTAs per SM (24
+// warps) when CH <= 4 and 2 (16 warps, <= 128 registers) when CH = 8: more loads in flight at
+// small fan-in, where each element carries few bytes.
+template <int DT, int CH>
+__global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   __shared__ Bias s_bias;
   __shared__ int s_live;
   __shared__ float s_inv;
@@ -395,7 +399,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     unpack(ld_stream(sp + i), ld_stream(sp + i + 4), P);
     unpack(ld_stream(sm + i), ld_stream(sm + i + 4), M);
     unpack(ld_stream(sv + i), ld_stream(sv + i + 4), V);
-    fan_in8<DT>(a.grads, a.Nd, i, s);
+    fan_in8<DT, CH>(a.grads, a.Nd, i, s);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const float g = __fmul_rn(s[k], inv);
