@@ -57,9 +57,10 @@ extern "C" {
 /* zero_step flags */
 #define ZERO_FUSED 0     /* stages 1/2: one fused pass (default); state copies ping-pong */
 #define ZERO_TWO_PASS 1  /* stages 1/2: reduce-scatter into grad_shard, then Adam + all-gather */
-#define ZERO_NO_TMA 2    /* ZERO_FUSED: always use the register-pipelined kernel; stage 3: gather
-                            layers with the register kernel instead of the TMA fan-out */
-#define ZERO_FORCE_TMA 4 /* ZERO_FUSED: use the TMA-pipelined kernel whenever buffers are aligned */
+#define ZERO_NO_TMA 2    /* ZERO_FUSED: always use the register-pipelined kernel */
+#define ZERO_FORCE_TMA 4 /* ZERO_FUSED: use the TMA-pipelined kernel whenever buffers are aligned;
+                            stage 3: gather layers with the TMA fan-out instead of the register
+                            kernel (the default) */
 #define ZERO_BF16_GRAD_SHARD 8 /* ZERO_TWO_PASS / stage 3: keep the reduced gradient as bf16 (see
                                   grad_shard); not described by the pages */
 

@@ -707,12 +707,15 @@ def test_gather_layer_full(L, Nd, nout):
         assert u16(o).tobytes() == want.tobytes()
 
 
+@pytest.mark.parametrize("gather", ["register", "tma"])
 @pytest.mark.parametrize("layer_len,N,Nd", [(1000, 5333, 3), (4096, 4096 * 3, 8),
-                                            (12_345, 12_345 * 2 + 17, 4)])
-def test_zero3_step_matches_oracle(layer_len, N, Nd):
-    """zero_step(stage=3): per-layer gather from the bf16 shards, per-layer reduce-scatter,
-    then Adam on every shard and the bf16 shard update; three steps, every element."""
-    buf = zero.ZeroBuffers(3, Nd, N, layer_len=layer_len, per_layer_buffers=True)
+                                            (12_345, 12_345 * 2 + 17, 4), (65_536, 65_536 * 3, 8)])
+def test_zero3_step_matches_oracle(layer_len, N, Nd, gather):
+    """zero_step(stage=3): per-layer gather from the bf16 shards (register kernel, or the TMA
+    fan-out with ZERO_FORCE_TMA), per-layer reduce-scatter, then Adam on every shard and the
+    bf16 shard update; three steps, every element."""
+    flags = zero.ZERO_FORCE_TMA if gather == "tma" else zero.ZERO_FUSED
+    buf = zero.ZeroBuffers(3, Nd, N, flags=flags, layer_len=layer_len, per_layer_buffers=True)
     sizes = buf.layer_sizes
     hp = dict(HP_ADAMW_ZERO3)
     total = buf.Np
