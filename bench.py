@@ -76,9 +76,12 @@ WORKLOADS = {
 DEFAULT = "zero1-gpt2-small"
 
 
-def bytes_per_param(w, two_pass=False, g16=False) -> int:
+def bytes_per_param(w, two_pass=False, g16=False, fused_layers=False) -> int:
     Nd = w["Nd"]
     gb = 2 if g16 else 4  # bytes of the kept reduced gradient
+    if w["stage"] == 3 and fused_layers:
+        # gather: 2 read + 2Nd written; fused pass: 2Nd + 12 read, 12 + 2 (bf16 shard) written
+        return (2 + 2 * Nd) + (2 * Nd + 12 + 12 + 2)
     if w["stage"] == 3:
         # gather: 2 read + 2Nd written; RS: 2Nd read + gb written; Adam + cast: gb + 24 + 2
         return (2 + 2 * Nd) + (2 * Nd + gb) + (gb + 24 + 2)
@@ -409,6 +412,8 @@ def main():
                     help="two-pass / stage 3: keep the reduced gradient as bf16")
     ap.add_argument("--two-pass", action="store_true",
                     help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather")
+    ap.add_argument("--fused-layers", action="store_true",
+                    help="stage 3: one speculative fused pass per layer (two fp32 state copies)")
     ap.add_argument("--bucket-override", type=int, default=-1,
                     help="stages 1/2: run with a different bucket size (0 = one bucket)")
     ap.add_argument("--nd-override", type=int, default=0,
@@ -438,8 +443,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     config = {"workload": w["desc"], "N": w["N"], "Nd": w["Nd"], "stage": w["stage"],
               "bucket": w["bucket"], "grad_dtype": w["gdt"], "state_dtype": "f32",
-              "path": ("two-pass" if args.two_pass else ("per-layer" if w["stage"] == 3 else
-                                                          "fused"))
+              "path": ("two-pass" if args.two_pass else
+                       ("per-layer fused" if w["stage"] == 3 and args.fused_layers else
+                        ("per-layer" if w["stage"] == 3 else "fused")))
               + (", bf16 gradient shard" if args.bf16_grad_shard else ""),
               "weights_dtype": "bf16", "parallelism": "replicas (%d simulated ranks per GPU)"
               % w["Nd"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
@@ -503,7 +509,9 @@ def main():
     # which fused kernel zero_step picks (mirrors the library's rule)
     tma_path = (not args.two_pass and w["stage"] != 3 and not args.no_tma and
                 (args.tma or (w["Nd"] >= 32 and (w["bucket"] or w["N"]) >= (1 << 26))))
-    if w["stage"] == 3:
+    if w["stage"] == 3 and args.fused_layers:
+        line_kernel = "zero3 step: gather_layer + fused_step kernels (per layer)"
+    elif w["stage"] == 3:
         line_kernel = "zero3 step: gather_layer + reduce_scatter + adam kernels"
     elif args.two_pass:
         line_kernel = "reduce_scatter + adam kernels (two-pass)"
@@ -516,7 +524,8 @@ def main():
         assert w["layer"] % Nd == 0 and N % w["layer"] == 0, "unpadded layers expected"
         buf = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, layer_len=w["layer"],
                                flags=(zero.ZERO_BF16_GRAD_SHARD if args.bf16_grad_shard else 0)
-                               | (zero.ZERO_NO_TMA if args.no_tma else 0))
+                               | (zero.ZERO_FORCE_TMA if args.tma else 0)
+                               | (zero.ZERO_FUSED_LAYERS if args.fused_layers else 0))
     else:
         buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt, flags=flags)
     glen = buf.grads[0].numel()  # N (stages 1/2) or one layer (stage 3, reused per layer)
@@ -547,7 +556,9 @@ def main():
             st.grads[r] = gs[r].data_ptr()
         states.append(st)
     nb = 1 if w["bucket"] == 0 else -(-N // w["bucket"])
-    if stage == 3:
+    if stage == 3 and args.fused_layers:
+        launches_per_step = 2 * nb + 1  # per layer: gather, fused pass; the overflow-repair check
+    elif stage == 3:
         launches_per_step = 3 * nb  # per layer: gather, reduce-scatter, Adam
     elif args.two_pass:
         launches_per_step = 2 * nb  # per bucket: reduce-scatter, Adam + all-gather
@@ -593,7 +604,7 @@ def main():
     ms_total, kern_ms = max_over_ranks([ms_total, kern_ms], dist, dev)
     ms_step = ms_total / args.steps
     value = whole_job_rate(N, world, ms_step)
-    bpp = bytes_per_param(w, args.two_pass, args.bf16_grad_shard)
+    bpp = bytes_per_param(w, args.two_pass, args.bf16_grad_shard, args.fused_layers)
     achieved = bpp * N / (kern_ms / 1e3) / 1e9
     peak, peak_src = peaks()
     tr = None

@@ -63,6 +63,10 @@ extern "C" {
                             kernel (the default) */
 #define ZERO_BF16_GRAD_SHARD 8 /* ZERO_TWO_PASS / stage 3: keep the reduced gradient as bf16 (see
                                   grad_shard); not described by the pages */
+#define ZERO_FUSED_LAYERS 16   /* stage 3: one fused pass per layer (reduce-scatter + AdamW + bf16
+                                  shard) writing the other state copy, speculatively, as ZERO_FUSED
+                                  does for stages 1/2; needs both state copies, no grad_shard, no
+                                  clipping; same results (see zero_step) */
 
 /* zero_allgather gates */
 #define ZERO_GATE_ALWAYS 0      /* always cast and write */
@@ -102,7 +106,8 @@ typedef struct {
     int64_t step;       /* completed (not skipped) updates t */
     int64_t skipped;    /* steps skipped because of an overflow */
     int32_t overflow;   /* 1 if the last finished step was skipped */
-    int32_t live;       /* ZERO_FUSED: index (0/1) of the state copy that holds the current state */
+    int32_t live;       /* ZERO_FUSED / ZERO_FUSED_LAYERS: index (0/1) of the state copy that
+                           holds the current state */
     double grad_sumsq;  /* sum of squares of the last finished step's reduced gradient */
     int32_t pending_overflow; /* overflow accumulated by the step in progress */
     int32_t reserved;
@@ -121,7 +126,7 @@ typedef struct {
  * Unused fields may be NULL. */
 typedef struct {
     int32_t grad_dtype;  /* ZERO_BF16 or ZERO_FP16 */
-    int32_t flags;       /* ZERO_FUSED or ZERO_TWO_PASS (stages 1/2) */
+    int32_t flags;       /* ZERO_FUSED or ZERO_TWO_PASS (stages 1/2), plus the ZERO_* options */
     /* stages 1/2: rank r's gradient replica (N elements) and bf16 weight replica (N elements).
      * stage 3: rank r's gradient buffer and gathered-weight buffer for the layer being
      * processed; layer l uses grads[r] + l*grad_layer_stride and params[r] + l*param_layer_stride
@@ -129,12 +134,14 @@ typedef struct {
     const uint16_t *grads[ZERO_MAX_ND];
     uint16_t *params[ZERO_MAX_ND];
     /* fp32 state, each padded (stages 1/2: Nd*S floats; stage 3: the padded layers back to back).
-     * ZERO_FUSED reads copy `live` and writes copy 1-live, so both copies must be allocated and
-     * zero-initialised in their padding; the other paths use copy 0 in place. */
+     * ZERO_FUSED (stages 1/2) and ZERO_FUSED_LAYERS (stage 3) read copy `live` and write copy
+     * 1-live, so both copies must be allocated and zero-initialised in their padding; the other
+     * paths use copy 0 in place. */
     float *master[2];
     float *exp_avg[2];
     float *exp_avg_sq[2];
-    float *grad_shard;      /* reduced gradient, same padded length (ZERO_TWO_PASS, stage 3): fp32,
+    float *grad_shard;      /* reduced gradient, same padded length (ZERO_TWO_PASS, stage 3 without
+                               ZERO_FUSED_LAYERS): fp32,
                                or bf16 (uint16_t storage, cast to float*) with ZERO_BF16_GRAD_SHARD:
                                the reduced mean is then rounded to bf16 (nearest even) before it is
                                stored, and the overflow check, the norm and the update use the
@@ -254,6 +261,14 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
  *     weights from param_shard into params[r] (every rank), reduce-scatter its gradient
  *     replicas into grad_shard; after the last layer, if no overflow, Adam in place on copy 0
  *     and param_shard = bf16(master).
+ *   stage 3, ZERO_FUSED_LAYERS: for each layer, the gather as above, then one fused pass over
+ *     the layer (reduce-scatter of its gradient replicas, unscale, overflow check, Adam from
+ *     copy `live` into copy 1-live, and the layer's param_shard = bf16(new master)).  The
+ *     overflow decision needs every layer, so the updates are speculative: the end of the step
+ *     swaps the copies if no element overflowed; otherwise param_shard is rewritten from the
+ *     unchanged copy.  Same values as the two-phase stage 3, 28 + 4*Nd bytes of traffic per
+ *     parameter instead of 36 + 4*Nd, for a second fp32 state copy (12 bytes per parameter);
+ *     no grad_shard; refuses max_grad_norm > 0 and ZERO_BF16_GRAD_SHARD (ZERO_EINVAL).
  * Every path skips the whole update (state, weights, t) when any reduced gradient element is
  * inf or NaN.  Asynchronous: call zero_read_result to learn whether the step was skipped. */
 int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t *st,

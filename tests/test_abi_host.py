@@ -131,6 +131,33 @@ def test_fused_step_refuses_clipping(zero):
     assert "ZERO_BF16_GRAD_SHARD" in str(e.value)
 
 
+def test_fused_layers_refusals(zero):
+    """Stage 3 with ZERO_FUSED_LAYERS: clipping, a bf16 gradient shard or a missing second state
+    copy are refused before any device work."""
+    st = zero.zero_state_t()
+    st.grad_dtype = zero.ZERO_BF16
+    st.flags = zero.ZERO_FUSED_LAYERS
+    for r in range(4):  # fake, never dereferenced
+        st.grads[r] = 4096
+        st.params[r] = 4096
+    for k in range(2):
+        st.master[k] = st.exp_avg[k] = st.exp_avg_sq[k] = 4096
+    st.param_shard = 4096
+    st.workspace = 4096
+    with pytest.raises(zero.ZeroError) as e:
+        zero.zero_step(3, 4, 1000, 500, st, zero.hparams(1e-3, max_grad_norm=1.0))
+    assert e.value.code == zero.ZERO_EINVAL and "clip" in str(e.value)
+    st.flags = zero.ZERO_FUSED_LAYERS | zero.ZERO_BF16_GRAD_SHARD
+    with pytest.raises(zero.ZeroError) as e:
+        zero.zero_step(3, 4, 1000, 500, st, zero.hparams(1e-3))
+    assert "ZERO_BF16_GRAD_SHARD" in str(e.value)
+    st.flags = zero.ZERO_FUSED_LAYERS
+    st.master[1] = 0
+    with pytest.raises(zero.ZeroError) as e:
+        zero.zero_step(3, 4, 1000, 500, st, zero.hparams(1e-3))
+    assert "both state copies" in str(e.value)
+
+
 def test_offload_step_validates_before_touching_the_device(zero):
     hp = zero.hparams(1e-3)
     st = zero.zero_offload_state_t()

@@ -537,7 +537,8 @@ def test_randomized_against_oracle(case):
 # ----------------------------------------------------------------------------- CUDA graphs
 
 @pytest.mark.parametrize("stage,flags", [(2, zero.ZERO_FUSED), (2, zero.ZERO_FUSED | zero.ZERO_FORCE_TMA),
-                                         (2, zero.ZERO_TWO_PASS), (3, zero.ZERO_FUSED)])
+                                         (2, zero.ZERO_TWO_PASS), (3, zero.ZERO_FUSED),
+                                         (3, zero.ZERO_FUSED_LAYERS)])
 def test_step_captured_in_a_cuda_graph_matches_eager(stage, flags):
     """The whole step is device-resident (step counter, live copy, overflow decision and loss
     scale live in the workspace), so it can be captured once and replayed: three replays with
@@ -546,8 +547,8 @@ def test_step_captured_in_a_cuda_graph_matches_eager(stage, flags):
     hp = zero.hparams(lr=1e-3, weight_decay=0.01)
     outs = []
     for use_graph in (False, True):
-        buf = (zero.ZeroBuffers(3, Nd, N, layer_len=L, per_layer_buffers=True) if stage == 3
-               else zero.ZeroBuffers(stage, Nd, N, flags=flags))
+        buf = (zero.ZeroBuffers(3, Nd, N, flags=flags, layer_len=L, per_layer_buffers=True)
+               if stage == 3 else zero.ZeroBuffers(stage, Nd, N, flags=flags))
         fill(buf.master[0], synth.NORMAL, synth.F32, synth.MASTER_STREAM, n=N, sigma=0.02)
         buf.init_workspace(0)
         buf.sync_params_from_master()
@@ -707,14 +708,17 @@ def test_gather_layer_full(L, Nd, nout):
         assert u16(o).tobytes() == want.tobytes()
 
 
-@pytest.mark.parametrize("gather", ["register", "tma"])
+@pytest.mark.parametrize("path", ["register-gather", "tma-gather", "fused-layers"])
 @pytest.mark.parametrize("layer_len,N,Nd", [(1000, 5333, 3), (4096, 4096 * 3, 8),
                                             (12_345, 12_345 * 2 + 17, 4), (65_536, 65_536 * 3, 8)])
-def test_zero3_step_matches_oracle(layer_len, N, Nd, gather):
+def test_zero3_step_matches_oracle(layer_len, N, Nd, path):
     """zero_step(stage=3): per-layer gather from the bf16 shards (register kernel, or the TMA
     fan-out with ZERO_FORCE_TMA), per-layer reduce-scatter, then Adam on every shard and the
-    bf16 shard update; three steps, every element."""
-    flags = zero.ZERO_FORCE_TMA if gather == "tma" else zero.ZERO_FUSED
+    bf16 shard update -- or, with ZERO_FUSED_LAYERS, one speculative fused pass per layer into
+    the other state copy; four steps, the third overflowing (+inf in one replica of the last
+    layer), every element."""
+    flags = {"register-gather": zero.ZERO_FUSED, "tma-gather": zero.ZERO_FORCE_TMA,
+             "fused-layers": zero.ZERO_FUSED_LAYERS}[path]
     buf = zero.ZeroBuffers(3, Nd, N, flags=flags, layer_len=layer_len, per_layer_buffers=True)
     sizes = buf.layer_sizes
     hp = dict(HP_ADAMW_ZERO3)
@@ -732,12 +736,14 @@ def test_zero3_step_matches_oracle(layer_len, N, Nd, gather):
     sh16 = oracle.f32_to_bf16(om)
     assert u16(buf.param_shard).tobytes() == sh16.tobytes()
     t = 0
-    for k in (1, 2, 3):
+    for k in (1, 2, 3, 4):
         hgrads, gathered = [], []
         for l, Ll in enumerate(sizes):
             for r in range(Nd):
                 hg = synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(k, r, l),
                                      Ll, sigma=1e-3)
+                if k == 3 and l == len(sizes) - 1 and r == Nd - 1:
+                    hg[Ll // 2] = 0x7F80  # +inf: the whole step is skipped
                 hgrads.append(hg)
                 buf.grads[r][l * layer_len:l * layer_len + Ll].view(torch.int16).copy_(
                     torch.from_numpy(hg.view(np.int16)))
@@ -749,12 +755,17 @@ def test_zero3_step_matches_oracle(layer_len, N, Nd, gather):
             for r in range(Nd):
                 got = u16(buf.params[r][l * layer_len:l * layer_len + Ll])
                 assert got.tobytes() == gathered[l * Nd + r].tobytes(), "gather layer %d" % l
+        if k == 3:
+            assert buf.result()["overflow"] == 1 and buf.result()["skipped"] == 1
+            assert u16(buf.param_shard).tobytes() == sh16.tobytes(), "skipped step changed shards"
     res = buf.result()
-    assert res["step"] == t == 3
+    assert res["step"] == t == 3 and res["skipped"] == 1
     assert abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
-    assert_f32_close(f32(buf.master[0]), om, "zero3 master")
-    assert_f32_close(f32(buf.exp_avg[0]), mm, "zero3 exp_avg")
-    assert_f32_close(f32(buf.exp_avg_sq[0]), vm, "zero3 exp_avg_sq")
+    live = buf.live()
+    assert live == (1 if path == "fused-layers" else 0)  # three committed flips
+    assert_f32_close(f32(buf.master[live]), om, "zero3 master")
+    assert_f32_close(f32(buf.exp_avg[live]), mm, "zero3 exp_avg")
+    assert_f32_close(f32(buf.exp_avg_sq[live]), vm, "zero3 exp_avg_sq")
     assert_bf16_close(u16(buf.param_shard), sh16, "zero3 bf16 shard")
     del buf
     free()

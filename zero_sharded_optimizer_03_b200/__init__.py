@@ -23,7 +23,7 @@ __all__ = [
     "ZeroOffloadBuffers",
     "zero_reduce_scatter_noalloc", "ZERO_NOALLOC_MAX_WINDOW", "hparams", "ZeroBuffers",
     "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_NO_TMA",
-    "ZERO_FORCE_TMA", "ZERO_BF16_GRAD_SHARD",
+    "ZERO_FORCE_TMA", "ZERO_BF16_GRAD_SHARD", "ZERO_FUSED_LAYERS",
     "ZERO_GATE_ALWAYS",
     "ZERO_GATE_NO_OVERFLOW", "ZERO_MAX_ND",
 ]
@@ -34,6 +34,7 @@ ZERO_OK, ZERO_EINVAL, ZERO_ECUDA = 0, -1, -2
 ZERO_MAX_ND = 64
 ZERO_BF16, ZERO_FP16 = 0, 1
 ZERO_FUSED, ZERO_TWO_PASS, ZERO_NO_TMA, ZERO_FORCE_TMA, ZERO_BF16_GRAD_SHARD = 0, 1, 2, 4, 8
+ZERO_FUSED_LAYERS = 16
 ZERO_GATE_ALWAYS, ZERO_GATE_NO_OVERFLOW = 0, 1
 
 _i64, _i32, _dbl, _P = ctypes.c_int64, ctypes.c_int32, ctypes.c_double, ctypes.c_void_p
@@ -345,11 +346,13 @@ class ZeroBuffers:
             self.grads = [torch.zeros(max(nbuf, 1), dtype=gdt, device=device) for _ in range(Nd)]
             self.params = [torch.zeros(max(nbuf, 1), dtype=torch.bfloat16, device=device)
                            for _ in range(Nd)]
-            self.master = [torch.zeros(self.Np, **f32)]
-            self.exp_avg = [torch.zeros(self.Np, **f32)]
-            self.exp_avg_sq = [torch.zeros(self.Np, **f32)]
+            fused = bool(flags & ZERO_FUSED_LAYERS)  # two state copies, no gradient shard
+            copies = 2 if fused else 1
+            self.master = [torch.zeros(self.Np, **f32) for _ in range(copies)]
+            self.exp_avg = [torch.zeros(self.Np, **f32) for _ in range(copies)]
+            self.exp_avg_sq = [torch.zeros(self.Np, **f32) for _ in range(copies)]
             gs_dt = torch.bfloat16 if flags & ZERO_BF16_GRAD_SHARD else torch.float32
-            self.grad_shard = torch.zeros(self.Np, dtype=gs_dt, device=device)
+            self.grad_shard = None if fused else torch.zeros(self.Np, dtype=gs_dt, device=device)
             self.param_shard = torch.zeros(self.Np, dtype=torch.bfloat16, device=device)
             st.grad_layer_stride = stride
             st.param_layer_stride = stride
@@ -382,8 +385,12 @@ class ZeroBuffers:
         return zero_read_result(self.ws.data_ptr(), self.stream())
 
     def live(self) -> int:
-        fused = not (self.flags & ZERO_TWO_PASS)
-        return self.result()["live"] if fused and self.stage in (1, 2) else 0
+        """Index of the state copy holding the current state (0 on the in-place paths)."""
+        if self.stage in (1, 2):
+            fused = not (self.flags & ZERO_TWO_PASS)
+        else:
+            fused = bool(self.flags & ZERO_FUSED_LAYERS)
+        return self.result()["live"] if fused else 0
 
     def sync_params_from_master(self) -> None:
         """Write bf16(master) into every weight replica (stage 1/2) or the bf16 shards
@@ -393,7 +400,7 @@ class ZeroBuffers:
             zero_allgather(self.master[live].data_ptr(), [p.data_ptr() for p in self.params],
                            self.Nd, 0, self.N, ZERO_GATE_ALWAYS, None, self.stream())
         else:
-            zero_allgather(self.master[0].data_ptr(), [self.param_shard.data_ptr()], 1, 0,
+            zero_allgather(self.master[live].data_ptr(), [self.param_shard.data_ptr()], 1, 0,
                            self.Np, ZERO_GATE_ALWAYS, None, self.stream())
 
 

@@ -390,6 +390,92 @@ void adam_host(float* p, float* m, float* v, const float* g, uint16_t* out16, in
 float clip_factor(double max_norm, double sumsq);
 }  // namespace zh
 
+// ZeRO-3 step with one fused pass per layer (flag ZERO_FUSED_LAYERS): the forward gather of
+// layer l, then the layer's reduce-scatter, unscale, flag / sum of squares, AdamW and bf16 cast
+// in one kernel (the K1 kernel with a single bf16 output: the layer's concatenated shards).  The
+// global overflow decision is known only after the last layer, so every layer's update goes into
+// the other state copy (read `live`, write 1 - live) and the bf16 shards are written
+// speculatively; the last layer's launch ends the step and makes the new copy live unless the
+// step overflowed, and an overflowed step has its bf16 shards rewritten from the unchanged live
+// copy.  Same arithmetic, same results as the two-phase stage 3 (no reduced-gradient shard), at
+// 28 + 4 Nd bytes per parameter instead of 36 + 4 Nd, for twice the fp32 state.
+static int zero3_fused_layers(int Nd, int64_t N, int64_t bucket, const zero_state_t* st, const zero_hparams_t* hp,
+                              const zb::Consts& c, cudaStream_t s) {
+  if (hp->max_grad_norm > 0)
+    return fail(ZERO_EINVAL,
+                "ZERO_FUSED_LAYERS cannot clip (the update would need the whole gradient's norm first): "
+                "use the two-phase stage 3");
+  if (st->flags & ZERO_BF16_GRAD_SHARD)
+    return fail(ZERO_EINVAL, "ZERO_FUSED_LAYERS keeps no reduced-gradient shard (ZERO_BF16_GRAD_SHARD)");
+  for (int i = 0; i < 2; ++i)
+    if (!st->master[i] || !st->exp_avg[i] || !st->exp_avg_sq[i])
+      return fail(ZERO_EINVAL, "ZERO_FUSED_LAYERS needs both state copies (master/exp_avg/exp_avg_sq [0] and [1])");
+  if (!st->param_shard) return fail(ZERO_EINVAL, "stage 3 needs param_shard");
+  bool al = true;
+  int rc = check_ptrs(st->grads, Nd, "grads", &al);
+  if (rc) return rc;
+  if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
+  void* ws = st->workspace;
+  const int64_t L = bucket > 0 ? bucket : N;
+  const int64_t nl = (N + L - 1) / L;
+  prof_mark(true, s);
+  int64_t off = 0;
+  for (int64_t l = 0; l < nl; ++l) {
+    const int64_t Ll = (l + 1) * L <= N ? L : N - l * L;
+    const int64_t Sl = (Ll + Nd - 1) / Nd;
+    const uint16_t* shards[ZERO_MAX_ND];
+    uint16_t* outs[ZERO_MAX_ND];
+    for (int r = 0; r < Nd; ++r) {
+      shards[r] = st->param_shard + off + r * Sl;
+      outs[r] = st->params[r] + l * st->param_layer_stride;
+    }
+    rc = (st->flags & ZERO_FORCE_TMA) ? do_gather_tma(shards, Nd, Ll, outs, Nd, ws, s)
+                                      : do_gather(shards, Nd, Ll, outs, Nd, s);
+    if (rc) return rc;
+    zb::FusedArgs a;
+    std::memset(&a, 0, sizeof a);
+    bool fal = true;
+    for (int r = 0; r < Nd; ++r) {
+      a.grads[r] = st->grads[r] + l * st->grad_layer_stride;
+      fal = fal && aligned16(a.grads[r]);
+    }
+    a.reps[0] = st->param_shard + off;
+    a.nrep = 1;
+    for (int i = 0; i < 2; ++i) {  // the layer's slice of each state copy, indexed from the layer start
+      a.p[i] = st->master[i] + off;
+      a.m[i] = st->exp_avg[i] + off;
+      a.v[i] = st->exp_avg_sq[i] + off;
+      fal = fal && aligned16(a.p[i]) && aligned16(a.m[i]) && aligned16(a.v[i]);
+    }
+    fal = fal && aligned16(a.reps[0]);
+    a.lo = 0;
+    a.hi = Ll;
+    a.c = c;
+    a.hdr = header(ws);
+    a.part = partials(ws);
+    a.Nd = Nd;
+    a.vec = fal;
+    a.mode = (l == 0 ? zb::kAccSet : zb::kAccAdd) | (l == nl - 1 ? (zb::kFinalize | zb::kFlip) : 0);
+    if ((rc = launch_fused(st->grad_dtype, a, s))) return rc;
+    off += Sl * Nd;
+  }
+  prof_mark(false, s);
+  // overflow repair: the bf16 shards from the unchanged live copy (runs only after a skip); the
+  // shards and the state share one padded layout, so one launch covers every layer
+  zb::CastArgs r;
+  std::memset(&r, 0, sizeof r);
+  r.src[0] = st->master[0];
+  r.src[1] = st->master[1];
+  r.reps[0] = st->param_shard;
+  r.nrep = 1;
+  r.gate = zb::kGateRepair;
+  r.lo = 0;
+  r.hi = off;
+  r.hdr = header(ws);
+  r.vec = aligned16(r.src[0]) && aligned16(r.src[1]) && aligned16(r.reps[0]);
+  return launch_cast(r, s);
+}
+
 // ==================================================================== C ABI
 
 extern "C" {
@@ -588,6 +674,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     return launch_ws(ws, zb::kWsEnd, 0, s);
   }
 
+  if (stage == 3 && (st->flags & ZERO_FUSED_LAYERS)) return zero3_fused_layers(Nd, N, bucket, st, hp, c, s);
   if (stage == 3) {
     if (!st->master[0] || !st->exp_avg[0] || !st->exp_avg_sq[0] || !st->grad_shard || !st->param_shard)
       return fail(ZERO_EINVAL, "stage 3 needs master[0], exp_avg[0], exp_avg_sq[0], grad_shard, param_shard");
@@ -756,6 +843,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   a.hdr = header(ws);
   a.part = partials(ws);
   a.Nd = Nd;
+  a.nrep = Nd;
   a.vec = al;
   // The TMA pipeline wins only where many loads must be in flight per element: a wide fan-in
   // over a long window (measured on B200: +1.2% at Nd = 64 over 2^28 elements; -1..-3% at
@@ -1131,6 +1219,7 @@ extern "C" int zero_fused_window(int Nd, int64_t lo, int64_t hi, const zero_stat
   a.hdr = header(st->workspace);
   a.part = partials(st->workspace);
   a.Nd = Nd;
+  a.nrep = Nd;
   a.vec = al;
   a.lo = lo;
   a.hi = hi;

@@ -362,7 +362,7 @@ struct FusedArgs {
   int Nd;
   int mode;
   int vec;
-  int unused;
+  int nrep;  // bf16 outputs per element: the Nd replicas (ZeRO-1/2), or 1 (a ZeRO-3 layer's shard)
 };
 
 // CH: gradient replicas loaded per batch (1, 2, 4 or 8).  Built for 3 resident CTAs per SM (24
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
     st_stream(dv + i, make_float4(V[0], V[1], V[2], V[3]));
     st_stream(dv + i + 4, make_float4(V[4], V[5], V[6], V[7]));
     const uint4 w = pack_bf16x8(P);
-    for (int r = 0; r < a.Nd; ++r) st_stream(a.reps[r] + i, w);
+    for (int r = 0; r < a.nrep; ++r) st_stream(a.reps[r] + i, w);
   }
   for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
     const int64_t i = sp8.scalar_index(a.lo, e);
@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
     dm[i] = M;
     dv[i] = V;
     const uint16_t w = to_bf16(P);
-    for (int r = 0; r < a.Nd; ++r) a.reps[r][i] = w;
+    for (int r = 0; r < a.nrep; ++r) a.reps[r][i] = w;
   }
   block_finish(sq, bad, a.hdr, a.part, a.mode);
 }
