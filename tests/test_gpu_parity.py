@@ -534,6 +534,85 @@ def test_randomized_against_oracle(case):
     free()
 
 
+def _random_zero3_cases(n_cases=24, seed=2027):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for k in range(n_cases):
+        Nd = int(rng.choice([1, 2, 3, 4, 5, 8, 13, 16]))
+        L = int(rng.choice([1, 7, 1000, 4096, 4097, 20_000, 65_536, 65_541]))
+        nl = int(rng.integers(1, 5))
+        N = L * nl - int(rng.integers(0, L)) if nl > 1 else L  # the last layer may be shorter
+        gdt = int(rng.choice([zero.ZERO_BF16, zero.ZERO_FP16]))
+        path = ["two-phase", "two-phase-g16", "tma-gather", "fused-layers"][k % 4]
+        clip = path.startswith("two-phase") and bool(rng.random() < 0.5)
+        dyn = bool(rng.random() < 0.3)
+        inject = bool(rng.random() < 0.25)
+        cases.append((k, N, L, Nd, gdt, path, clip, dyn, inject))
+    return cases
+
+
+@pytest.mark.parametrize("case", _random_zero3_cases(), ids=lambda c: "case%d" % c[0])
+def test_randomized_zero3_against_flat_oracle(case):
+    """Seeded random ZeRO-3 layer shapes, paths and options, three steps each: ZeRO-3 computes
+    what unsharded data parallelism computes, so every real element equals the flat oracle step
+    on the concatenated layers (state, bf16 shards, the next step's gathered weights)."""
+    k, N, L, Nd, gdt, path, clip, dyn, inject = case
+    odt, sdt = DT[gdt]
+    flags = {"two-phase": zero.ZERO_FUSED, "two-phase-g16": zero.ZERO_BF16_GRAD_SHARD,
+             "tma-gather": zero.ZERO_FORCE_TMA, "fused-layers": zero.ZERO_FUSED_LAYERS}[path]
+    max_norm = 1e-3 if clip else 0.0
+    ls = 64.0 if gdt == zero.ZERO_FP16 else 1.0
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=ls, max_grad_norm=max_norm,
+              bf16_grad=path == "two-phase-g16", dynamic_scale=dyn, scale_interval=1)
+    buf = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, flags=flags, layer_len=L,
+                           per_layer_buffers=True)
+    # real elements of the padded per-layer layout, in flat order
+    real = np.concatenate([np.arange(Ll) + sum(buf.layer_padded[:l])
+                           for l, Ll in enumerate(buf.layer_sizes)]).astype(np.int64)
+    om = synth.fill_host(synth.NORMAL, synth.F32, SEED, synth.MASTER_STREAM, N, sigma=0.02)
+    full = np.zeros(buf.Np, np.float32)
+    full[real] = om
+    buf.master[0].copy_(torch.from_numpy(full))
+    buf.init_workspace(0)
+    if dyn:
+        zero.zero_loss_scaler_init(buf.ws.data_ptr(), ls, 2.0, 0.5, 1, stream())
+    buf.sync_params_from_master()
+    _, Np, _ = oracle.partition(N, Nd)  # the flat oracle works on the flat padded layout
+    om = np.concatenate([om, np.zeros(Np - N, np.float32)])
+    mm = np.zeros(Np, np.float32)
+    vm = np.zeros(Np, np.float32)
+    oreps = [oracle.f32_to_bf16(om[:N]) for _ in range(Nd)]
+    t, scale, good = 0, ls, 0
+    for step in (1, 2, 3):
+        prev = oreps[0].copy()
+        sigma = float(np.float32(1e-3 * scale)) if gdt == zero.ZERO_FP16 else 1e-3
+        hg = [synth.fill_host(synth.NORMAL, sdt, SEED, synth.grad_stream(step, r), N, sigma=sigma)
+              for r in range(Nd)]
+        if inject and step == 2:
+            hg[Nd - 1][N // 2] = 0x7F80 if gdt == zero.ZERO_BF16 else 0x7C00  # +inf
+        for r in range(Nd):
+            buf.grads[r].view(torch.int16).copy_(torch.from_numpy(hg[r].view(np.int16)))
+        buf.step(zero.hparams(lr=1e-3, weight_decay=0.01, loss_scale=ls, max_grad_norm=max_norm))
+        t, ovf, ss, scale, good = oracle.zero12_step_ex(Nd, N, 0, odt, hg, om, mm, vm, oreps,
+                                                        hp, t, scale, good)
+        for r in range(Nd):  # the forward gather of this step saw the previous weights
+            assert u16(buf.params[r]).tobytes() == prev.tobytes(), "case %d gather" % k
+    res = buf.result()
+    assert res["step"] == t and res["skipped"] == (1 if inject else 0), (case, res)
+    if ss > 0 and np.isfinite(ss):
+        assert abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
+    if dyn:
+        assert res["loss_scale"] == scale
+    live = buf.live()
+    idx = torch.from_numpy(real).cuda()
+    assert_f32_close(f32(buf.master[live][idx]), om[:N], "case %d master" % k)
+    assert_f32_close(f32(buf.exp_avg[live][idx]), mm[:N], "case %d exp_avg" % k)
+    assert_f32_close(f32(buf.exp_avg_sq[live][idx]), vm[:N], "case %d exp_avg_sq" % k)
+    assert_bf16_close(u16(buf.param_shard[idx]), oreps[0], "case %d bf16 shard" % k)
+    del buf
+    free()
+
+
 # ----------------------------------------------------------------------------- CUDA graphs
 
 @pytest.mark.parametrize("stage,flags", [(2, zero.ZERO_FUSED), (2, zero.ZERO_FUSED | zero.ZERO_FORCE_TMA),
