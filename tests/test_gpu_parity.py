@@ -216,6 +216,45 @@ def test_tma_and_register_kernels_identical(Nd, gdt):
     free()
 
 
+# 64 vectors per thread of one wave: 148 SMs x 3 CTAs x 256 threads x 64 x 8 elements (1 to 4
+# replicas per batch), 148 x 2 x 256 x 64 x 8 (batches of 8)
+CHUNKED_MIN_N = {1: 58_195_968, 4: 58_195_968, 12: 38_797_312}
+
+
+@pytest.mark.parametrize("Nd,gdt,flags", [(1, zero.ZERO_BF16, zero.ZERO_NO_TMA),
+                                          (2, zero.ZERO_BF16, zero.ZERO_NO_TMA),
+                                          (4, zero.ZERO_FP16, zero.ZERO_NO_TMA),
+                                          (12, zero.ZERO_BF16, zero.ZERO_NO_TMA),
+                                          (16, zero.ZERO_FP16, zero.ZERO_FORCE_TMA)])
+def test_long_windows_match_oracle(Nd, gdt, flags):
+    """Windows long enough for the load-balanced schedules -- the fused kernel's dynamically
+    scheduled chunks (Nd = 1, 4, 12: just above the length that switches them on), its fixed
+    grid-stride split (Nd = 2) and the TMA kernel's multi-wave grid (Nd = 16: 16.4M elements,
+    3 waves) -- against the oracle at every element: two steps, a ragged tail."""
+    N = CHUNKED_MIN_N.get(Nd, 2048 * 8000) + 1237
+    odt, sdt = DT[gdt]
+    ls = 64.0 if gdt == zero.ZERO_FP16 else 1.0
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=ls)
+    buf = zero.ZeroBuffers(2, Nd, N, grad_dtype=gdt, flags=zero.ZERO_FUSED | flags)
+    _init_state(buf, N)
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    oreps = [oracle.f32_to_bf16(om[:N]) for _ in range(Nd)]
+    t = 0
+    for step in (1, 2):
+        sigma = float(np.float32(1e-3 * ls))
+        hg = [synth.fill_host(synth.NORMAL, sdt, SEED, synth.grad_stream(step, r), N, sigma=sigma)
+              for r in range(Nd)]
+        for r in range(Nd):
+            fill(buf.grads[r], synth.NORMAL, sdt, synth.grad_stream(step, r), sigma=sigma)
+        buf.step(zero.hparams(**hp))
+        t, ovf, ss = oracle.zero12_step(Nd, N, 0, odt, hg, om, mm, vm, oreps, hp, t)
+    res = _compare_full(buf, om, mm, vm, oreps, t, ss, "long window Nd=%d" % Nd)
+    assert res["error"] == 0 and res["skipped"] == 0
+    del buf
+    free()
+
+
 def test_stage1_and_stage2_identical():
     Nd, N = 8, 300_001
     outs = []

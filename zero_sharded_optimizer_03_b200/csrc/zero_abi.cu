@@ -110,13 +110,18 @@ int grid_for(int kid, int64_t work, int* grid, int waves = 1, bool partials = tr
   return ZERO_OK;
 }
 
-// Waves per kernel (see grid_for), from the same-box sweeps: fused kernel with 1 or 4 replicas
-// per batch and above 8 replicas: 4; with 2 or exactly 8: 1; reduce-scatter 4; in-place Adam 8;
-// layer gather 16 (it has no partials).
+// Waves per kernel (see grid_for), from the same-box sweeps: reduce-scatter 4, in-place Adam 8,
+// layer gather 16 (it has no partials).  The fused kernel balances its SMs with dynamically
+// scheduled chunks instead (use_chunks), and the TMA kernel with waves of its own (tma_grid).
 constexpr int kWavesRs = 4;
 constexpr int kWavesAdam = 8;
 constexpr int kWavesGather = 16;
-inline int fused_waves(int Nd) { return (Nd == 2 || (Nd >= 5 && Nd <= 8)) ? 1 : 4; }
+
+// Fused kernel over a long window: chunks handed out by the workspace counter, or the fixed
+// grid-stride split.  Same-box sweeps at 2^25-2^28 elements, chunks against the best fixed grid:
+// +15% at Nd = 1, +7% at Nd = 4, +4% at Nd = 16, +2% at Nd = 64; -2% at Nd = 2 and with a
+// single bf16 output (ZeRO-3 layers), +-1% at Nd = 8.
+inline bool use_chunks(int Nd, int nrep) { return nrep > 1 ? !(Nd == 2 || (Nd >= 5 && Nd <= 8)) : Nd == 1; }
 
 // SM count of the current device, and the TMA kernels' shared-memory attribute set once.
 int tma_setup(int* sms) {
@@ -236,10 +241,15 @@ void prof_mark(bool start, cudaStream_t s) {
 // ------------------------------------------------------------------ launchers
 
 template <int DT, int CH>
-int launch_fused_ch(int kid, const zb::FusedArgs& a, cudaStream_t s) {
+int launch_fused_ch(int kid, zb::FusedArgs a, cudaStream_t s) {
   int grid = 0;
-  int rc = grid_for(kid, (a.hi - a.lo + 7) / 8, &grid, fused_waves(a.Nd));
+  const int64_t work = (a.hi - a.lo + 7) / 8;
+  int rc = grid_for(kid, work, &grid);
   if (rc) return rc;
+  // chunks only for long windows (>= 64 vectors per thread of the wave: on the 25M-element
+  // buckets of a 1.3e9-parameter fp16 job at Nd = 16, 16 per thread, they measured 1% slower)
+  // and launches whose last CTA resets the counter (mode != 0)
+  a.chunked = a.mode != 0 && work >= 64 * (int64_t)grid * zb::kThreads && use_chunks(a.Nd, a.nrep);
   zb::fused_step_kernel<DT, CH><<<grid, zb::kThreads, 0, s>>>(a);
   return check_launch("fused_step_kernel launch");
 }
@@ -262,7 +272,16 @@ int launch_fused_tma(int dtype, zb::TmaArgs& a, cudaStream_t s) {
   a.tiles_lo = (a.lo + 7) & ~int64_t(7);
   if (a.tiles_lo > a.hi) a.tiles_lo = a.hi;
   a.ntiles = (a.hi - a.tiles_lo) / zb::kTile;
-  int64_t grid = a.ntiles < sms ? a.ntiles : sms;
+  // Several waves of one-CTA-per-SM blocks (at least 16 tiles per CTA, at most 32 waves) let the
+  // block scheduler give more tiles to the SMs that stream faster: same-box sweep at Nd = 64,
+  // 2^28 elements: 1 wave 6080 GB/s, 8 waves 6499, 16 6656, 32 6671; at Nd = 16, 1.3e9
+  // elements: 1 wave 5978, 16 waves 6635.
+  int64_t waves = a.ntiles / (16 * (int64_t)sms);
+  if (waves > 32) waves = 32;
+  if (waves < 1) waves = 1;
+  int64_t grid = (int64_t)sms * waves;
+  if (grid > zb::kMaxCtas) grid = zb::kMaxCtas;
+  if (grid > a.ntiles) grid = a.ntiles;
   if (grid < 1) grid = 1;
   a.stall_unit = g_test_stall;
   g_test_stall = -1;
@@ -845,10 +864,11 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   a.Nd = Nd;
   a.nrep = Nd;
   a.vec = al;
-  // The TMA pipeline wins only where many loads must be in flight per element: a wide fan-in
-  // over a long window (measured on B200: +1.2% at Nd = 64 over 2^28 elements; -1..-3% at
-  // Nd = 8..16, and a fixed cost per launch that hurts short bucketed windows).
-  const bool tma_auto = Nd >= 32 && B >= (int64_t(1) << 26);
+  // The TMA pipeline wins where many loads must be in flight per element over a long window
+  // (same box, with its multi-wave grid: Nd = 64, 2^28: 6671 GB/s against 6091 for the register
+  // kernel; Nd = 16, 1.3e9 in one bucket: 6635 against 6229); at Nd = 8 the two are equal, and
+  // a TMA launch has a fixed cost (~22 us) that hurts short bucketed windows.
+  const bool tma_auto = Nd >= 16 && B >= (int64_t(1) << 26);
   const bool tma = al && !(st->flags & ZERO_NO_TMA) && ((st->flags & ZERO_FORCE_TMA) || tma_auto);
   zb::TmaArgs ta;
   if (tma) {

@@ -47,6 +47,7 @@ struct Header {
   double growth, backoff; // scale factors after `interval` clean steps / after an overflow
   long long interval;
   long long good;         // clean steps since the last change of the scale
+  unsigned long long chunk;  // next work chunk of a dynamically scheduled launch (0 between launches)
 };
 static_assert(sizeof(Header) <= 256, "header must fit its slot");
 
@@ -214,6 +215,7 @@ template <int DT, int CH = 8>
 __device__ __forceinline__ void fan_in8(const uint16_t* const* grads, int Nd, int64_t i, float (&s)[8]) {
 #pragma unroll
   for (int k = 0; k < 8; ++k) s[k] = 0.0f;
+#pragma unroll 1
   for (int r0 = 0; r0 < Nd; r0 += CH) {
     uint4 q[CH];
 #pragma unroll
@@ -343,6 +345,7 @@ __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Pa
     }
     if (mode & kFinalize) end_step(hdr, mode & kFlip);
     hdr->done = 0u;
+    hdr->chunk = 0ull;  // every CTA has left its chunk loop: ready for the next launch
     __threadfence();
   }
 }
@@ -362,17 +365,31 @@ struct FusedArgs {
   int Nd;
   int mode;
   int vec;
-  int nrep;  // bf16 outputs per element: the Nd replicas (ZeRO-1/2), or 1 (a ZeRO-3 layer's shard)
+  int nrep;     // bf16 outputs per element: the Nd replicas (ZeRO-1/2), or 1 (a ZeRO-3 layer's shard)
+  int chunked;  // 1: CTAs take chunks of kChunkVecs vectors from hdr->chunk (needs mode != 0)
+  int unused;
 };
+
+// Vectors per dynamically scheduled chunk: 4 per thread of a CTA.
+constexpr int kChunkIters = 4;
+constexpr int64_t kChunkVecs = (int64_t)kChunkIters * kThreads;
 
 // CH: gradient replicas loaded per batch (1, 2, 4 or 8).  Built for 3 resident CTAs per SM (24
 // warps) when CH <= 4 and 2 (16 warps, <= 128 registers) when CH = 8: more loads in flight at
 // small fan-in, where each element carries few bytes.
+//
+// Work distribution: a grid-stride loop over one wave of resident CTAs (every SM owns a fixed
+// share of the window), or, with a.chunked, chunks of kChunkVecs vectors handed out by an atomic
+// counter in the workspace header, so that SMs that stream faster take more of the window; the
+// last CTA to finish resets the counter.  Which vector a thread updates does not change any
+// result (every element is independent); only the order in which the per-CTA sums of squares
+// are formed does.
 template <int DT, int CH>
 __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   __shared__ Bias s_bias;
   __shared__ int s_live;
   __shared__ float s_inv;
+  __shared__ long long s_chunk;
   if (threadIdx.x == 0) {
     s_bias = bias_for(a.c, __ldcg(&a.hdr->t) + 1);
     s_live = __ldcg(&a.hdr->live) & 1;
@@ -392,8 +409,9 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
   double sq = 0.0;
   int bad = 0;
   const Span sp8(a.lo, a.hi, a.vec);
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < sp8.nvec; j += stride) {
+  // one 8-element vector: Nd-way reduce-scatter, unscale, flag / sum of squares, AdamW from copy
+  // `live` into copy 1-live, bf16 cast fanned out to the nrep outputs
+  auto vector_step = [&](int64_t j) {
     const int64_t i = sp8.vlo + (j << 3);
     float P[8], M[8], V[8], s[8];
     unpack(ld_stream(sp + i), ld_stream(sp + i + 4), P);
@@ -415,7 +433,28 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
     st_stream(dv + i + 4, make_float4(V[4], V[5], V[6], V[7]));
     const uint4 w = pack_bf16x8(P);
     for (int r = 0; r < a.nrep; ++r) st_stream(a.reps[r] + i, w);
+  };
+  if (a.chunked) {
+    const int64_t nchunks = (sp8.nvec + kChunkVecs - 1) / kChunkVecs;
+    for (;;) {
+      if (threadIdx.x == 0) s_chunk = (long long)atomicAdd(&a.hdr->chunk, 1ull);
+      __syncthreads();
+      const int64_t c = s_chunk;
+      __syncthreads();  // every thread has read s_chunk before thread 0 takes the next one
+      if (c >= nchunks) break;
+      const int64_t j0 = c * kChunkVecs + threadIdx.x;
+#pragma unroll 1
+      for (int u = 0; u < kChunkIters; ++u) {
+        const int64_t j = j0 + (int64_t)u * kThreads;
+        if (j < sp8.nvec) vector_step(j);
+      }
+    }
+  } else {
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+#pragma unroll 1
+    for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < sp8.nvec; j += stride) vector_step(j);
   }
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
     const int64_t i = sp8.scalar_index(a.lo, e);
     const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), inv);
@@ -697,6 +736,7 @@ __global__ void ws_ctl_kernel(Header* h, int op, long long t0) {
     h->backoff = 1.0;
     h->interval = 1;
     h->good = 0;
+    h->chunk = 0ull;
   }
   if (op == kWsInit || op == kWsBegin) {
     h->pending_flag = 0;
