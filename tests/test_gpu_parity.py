@@ -218,19 +218,21 @@ def test_tma_and_register_kernels_identical(Nd, gdt):
 
 # 64 vectors per thread of one wave: 148 SMs x 3 CTAs x 256 threads x 64 x 8 elements (1 to 4
 # replicas per batch), 148 x 2 x 256 x 64 x 8 (batches of 8)
-CHUNKED_MIN_N = {1: 58_195_968, 4: 58_195_968, 12: 38_797_312}
+CHUNKED_MIN_N = {1: 58_195_968, 6: 58_195_968, 8: 58_195_968, 12: 38_797_312}
 
 
 @pytest.mark.parametrize("Nd,gdt,flags", [(1, zero.ZERO_BF16, zero.ZERO_NO_TMA),
                                           (2, zero.ZERO_BF16, zero.ZERO_NO_TMA),
-                                          (4, zero.ZERO_FP16, zero.ZERO_NO_TMA),
+                                          (6, zero.ZERO_FP16, zero.ZERO_NO_TMA),
+                                          (8, zero.ZERO_BF16, zero.ZERO_NO_TMA),
                                           (12, zero.ZERO_BF16, zero.ZERO_NO_TMA),
                                           (16, zero.ZERO_FP16, zero.ZERO_FORCE_TMA)])
 def test_long_windows_match_oracle(Nd, gdt, flags):
     """Windows long enough for the load-balanced schedules -- the fused kernel's dynamically
-    scheduled chunks (Nd = 1, 4, 12: just above the length that switches them on), its fixed
-    grid-stride split (Nd = 2) and the TMA kernel's multi-wave grid (Nd = 16: 16.4M elements,
-    3 waves) -- against the oracle at every element: two steps, a ragged tail."""
+    scheduled chunks (Nd = 1, 6, 8 in batches of 4 replicas, 12 in batches of 8: just above the
+    length that switches them on), its fixed grid-stride split (Nd = 2) and the TMA kernel's
+    multi-wave grid (Nd = 16: 16.4M elements, 3 waves) -- against the oracle at every element:
+    two steps, a ragged tail."""
     N = CHUNKED_MIN_N.get(Nd, 2048 * 8000) + 1237
     odt, sdt = DT[gdt]
     ls = 64.0 if gdt == zero.ZERO_FP16 else 1.0

@@ -119,9 +119,10 @@ constexpr int kWavesGather = 16;
 
 // Fused kernel over a long window: chunks handed out by the workspace counter, or the fixed
 // grid-stride split.  Same-box sweeps at 2^25-2^28 elements, chunks against the best fixed grid:
-// +15% at Nd = 1, +7% at Nd = 4, +4% at Nd = 16, +2% at Nd = 64; -2% at Nd = 2 and with a
-// single bf16 output (ZeRO-3 layers), +-1% at Nd = 8.
-inline bool use_chunks(int Nd, int nrep) { return nrep > 1 ? !(Nd == 2 || (Nd >= 5 && Nd <= 8)) : Nd == 1; }
+// +15% at Nd = 1, +7% at Nd = 4 and, with batches of 4 replicas, +1.4% (124M) to +3.7% (2^28)
+// at Nd = 8, +4% at Nd = 16, +2% at Nd = 64; -2% at Nd = 2 and with a single bf16 output
+// (ZeRO-3 layers, nrep = 1 < Nd).
+inline bool use_chunks(int Nd, int nrep) { return nrep == Nd && Nd != 2; }
 
 // SM count of the current device, and the TMA kernels' shared-memory attribute set once.
 int tma_setup(int* sms) {
@@ -254,12 +255,14 @@ int launch_fused_ch(int kid, zb::FusedArgs a, cudaStream_t s) {
   return check_launch("fused_step_kernel launch");
 }
 
-// The rank batch width follows the fan-in: 1, 2, 4 replicas per batch for Nd <= 4, else 8.
+// The rank batch width follows the fan-in: 1 or 2 replicas per batch for Nd <= 2, 4 up to
+// Nd = 8 (at Nd = 8 two batches of 4 with 24 resident warps per SM beat one batch of 8 with 16:
+// +1.4% to +3.7% with chunks, +3.5% for a single output), else 8.
 int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s) {
   const bool f16 = dtype == ZERO_FP16;
   if (a.Nd <= 1) return f16 ? launch_fused_ch<1, 1>(kFusedFp16C1, a, s) : launch_fused_ch<0, 1>(kFusedBf16C1, a, s);
   if (a.Nd <= 2) return f16 ? launch_fused_ch<1, 2>(kFusedFp16C2, a, s) : launch_fused_ch<0, 2>(kFusedBf16C2, a, s);
-  if (a.Nd <= 4) return f16 ? launch_fused_ch<1, 4>(kFusedFp16C4, a, s) : launch_fused_ch<0, 4>(kFusedBf16C4, a, s);
+  if (a.Nd <= 8) return f16 ? launch_fused_ch<1, 4>(kFusedFp16C4, a, s) : launch_fused_ch<0, 4>(kFusedBf16C4, a, s);
   return f16 ? launch_fused_ch<1, 8>(kFusedFp16, a, s) : launch_fused_ch<0, 8>(kFusedBf16, a, s);
 }
 
