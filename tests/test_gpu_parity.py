@@ -656,13 +656,15 @@ def test_randomized_zero3_against_flat_oracle(case):
 
 # ----------------------------------------------------------------------------- CUDA graphs
 
-@pytest.mark.parametrize("stage,flags", [(2, zero.ZERO_FUSED), (2, zero.ZERO_FUSED | zero.ZERO_FORCE_TMA),
-                                         (2, zero.ZERO_TWO_PASS), (3, zero.ZERO_FUSED),
-                                         (3, zero.ZERO_FUSED_LAYERS)])
-def test_step_captured_in_a_cuda_graph_matches_eager(stage, flags):
+@pytest.mark.parametrize("stage,flags,bucket", [(2, zero.ZERO_FUSED, 0), (2, zero.ZERO_FUSED, 20_000),
+                                                (2, zero.ZERO_FUSED | zero.ZERO_FORCE_TMA, 0),
+                                                (2, zero.ZERO_TWO_PASS, 0), (3, zero.ZERO_FUSED, 0),
+                                                (3, zero.ZERO_FUSED_LAYERS, 0)])
+def test_step_captured_in_a_cuda_graph_matches_eager(stage, flags, bucket):
     """The whole step is device-resident (step counter, live copy, overflow decision and loss
     scale live in the workspace), so it can be captured once and replayed: three replays with
-    fresh gradients give the same bytes as three eager steps, including a skipped one."""
+    fresh gradients give the same bytes as three eager steps, including a skipped one (with
+    buckets: later buckets are programmatic dependent launches inside the graph)."""
     Nd, N, L = 4, 2048 * 40 + 8, 2048 * 10 + 2
     hp = zero.hparams(lr=1e-3, weight_decay=0.01)
     outs = []
@@ -680,14 +682,14 @@ def test_step_captured_in_a_cuda_graph_matches_eager(stage, flags):
             if k == 2:
                 put_bits(buf.grads[1], 5, 0x7F80)
             if not use_graph:
-                buf.step(hp)
+                buf.step(hp, bucket=bucket)
                 continue
             if graph is None:
                 side.wait_stream(torch.cuda.current_stream())
                 graph = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(graph, stream=side):
-                    zero.zero_step(buf.stage, Nd, N, buf.layer_len if stage == 3 else 0, buf.state,
-                                   hp, side.cuda_stream)
+                    zero.zero_step(buf.stage, Nd, N, buf.layer_len if stage == 3 else bucket,
+                                   buf.state, hp, side.cuda_stream)
                 torch.cuda.current_stream().wait_stream(side)
             graph.replay()  # capture does not run the work: every step comes from a replay
         torch.cuda.synchronize()

@@ -242,7 +242,7 @@ void prof_mark(bool start, cudaStream_t s) {
 // ------------------------------------------------------------------ launchers
 
 template <int DT, int CH>
-int launch_fused_ch(int kid, zb::FusedArgs a, cudaStream_t s) {
+int launch_fused_ch(int kid, zb::FusedArgs a, bool dependent, cudaStream_t s) {
   int grid = 0;
   const int64_t work = (a.hi - a.lo + 7) / 8;
   int rc = grid_for(kid, work, &grid);
@@ -251,19 +251,40 @@ int launch_fused_ch(int kid, zb::FusedArgs a, cudaStream_t s) {
   // buckets of a 1.3e9-parameter fp16 job at Nd = 16, 16 per thread, they measured 1% slower)
   // and launches whose last CTA resets the counter (mode != 0)
   a.chunked = a.mode != 0 && work >= 64 * (int64_t)grid * zb::kThreads && use_chunks(a.Nd, a.nrep);
-  zb::fused_step_kernel<DT, CH><<<grid, zb::kThreads, 0, s>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(zb::kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  // a later bucket of the same step may overlap the previous one's tail (fixed split only: the
+  // chunk counter is shared between launches)
+  if (dependent && !a.chunked) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, zb::fused_step_kernel<DT, CH>, a);
+  if (e != cudaSuccess) return cuda_fail(e, "fused_step_kernel launch");
   return check_launch("fused_step_kernel launch");
 }
 
 // The rank batch width follows the fan-in: 1 or 2 replicas per batch for Nd <= 2, 4 up to
 // Nd = 8 (at Nd = 8 two batches of 4 with 24 resident warps per SM beat one batch of 8 with 16:
 // +1.4% to +3.7% with chunks, +3.5% for a single output), else 8.
-int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s) {
+// dependent: a later bucket of the same step, launched right after the previous bucket's fused
+// kernel on the same stream (programmatic dependent launch).
+int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s, bool dependent = false) {
   const bool f16 = dtype == ZERO_FP16;
-  if (a.Nd <= 1) return f16 ? launch_fused_ch<1, 1>(kFusedFp16C1, a, s) : launch_fused_ch<0, 1>(kFusedBf16C1, a, s);
-  if (a.Nd <= 2) return f16 ? launch_fused_ch<1, 2>(kFusedFp16C2, a, s) : launch_fused_ch<0, 2>(kFusedBf16C2, a, s);
-  if (a.Nd <= 8) return f16 ? launch_fused_ch<1, 4>(kFusedFp16C4, a, s) : launch_fused_ch<0, 4>(kFusedBf16C4, a, s);
-  return f16 ? launch_fused_ch<1, 8>(kFusedFp16, a, s) : launch_fused_ch<0, 8>(kFusedBf16, a, s);
+  const bool d = dependent;
+  if (a.Nd <= 1)
+    return f16 ? launch_fused_ch<1, 1>(kFusedFp16C1, a, d, s) : launch_fused_ch<0, 1>(kFusedBf16C1, a, d, s);
+  if (a.Nd <= 2)
+    return f16 ? launch_fused_ch<1, 2>(kFusedFp16C2, a, d, s) : launch_fused_ch<0, 2>(kFusedBf16C2, a, d, s);
+  if (a.Nd <= 8)
+    return f16 ? launch_fused_ch<1, 4>(kFusedFp16C4, a, d, s) : launch_fused_ch<0, 4>(kFusedBf16C4, a, d, s);
+  return f16 ? launch_fused_ch<1, 8>(kFusedFp16, a, d, s) : launch_fused_ch<0, 8>(kFusedBf16, a, d, s);
 }
 
 // TMA-pipelined fused step over [a.lo, a.hi): whole tiles through the bulk-copy pipeline, the
@@ -900,7 +921,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       ta.hi = a.hi;
       ta.mode = a.mode;
       if ((rc = launch_fused_tma(st->grad_dtype, ta, s))) return rc;
-    } else if ((rc = launch_fused(st->grad_dtype, a, s))) {
+    } else if ((rc = launch_fused(st->grad_dtype, a, s, k > 0))) {
       return rc;
     }
   }

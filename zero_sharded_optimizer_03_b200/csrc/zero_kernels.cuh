@@ -370,6 +370,15 @@ struct FusedArgs {
   int unused;
 };
 
+// Programmatic dependent launch: a grid launched with programmatic stream serialization may
+// start while the previous grid in the stream finishes.  launch_dependents lets the next grid
+// start; wait blocks until the previous grid has completed and its memory is visible (it
+// returns at once for a grid launched without the attribute).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Vectors per dynamically scheduled chunk: 4 per thread of a CTA.
 constexpr int kChunkIters = 4;
 constexpr int64_t kChunkVecs = (int64_t)kChunkIters * kThreads;
@@ -384,6 +393,11 @@ constexpr int64_t kChunkVecs = (int64_t)kChunkIters * kThreads;
 // last CTA to finish resets the counter.  Which vector a thread updates does not change any
 // result (every element is independent); only the order in which the per-CTA sums of squares
 // are formed does.
+//
+// Consecutive buckets of one step may be launched as programmatic dependents (fixed split
+// only): the next bucket's CTAs start streaming while this one's last CTAs finish.  The header
+// fields read at the start (t, live, loss scale) change only when a step ends, and a dependent
+// grid waits for its predecessor before it touches the partials and the counters.
 template <int DT, int CH>
 __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   __shared__ Bias s_bias;
@@ -395,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
     s_live = __ldcg(&a.hdr->live) & 1;
     s_inv = step_inv(a.c, a.hdr);
   }
+  pdl_launch_dependents();
   __syncthreads();
   const Bias b = s_bias;
   const int live = s_live;
@@ -468,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
     const uint16_t w = to_bf16(P);
     for (int r = 0; r < a.nrep; ++r) a.reps[r][i] = w;
   }
+  pdl_wait();  // a programmatic dependent: the previous bucket has completed
   block_finish(sq, bad, a.hdr, a.part, a.mode);
 }
 
