@@ -508,7 +508,7 @@ def main():
         flags |= zero.ZERO_FORCE_TMA
     # which fused kernel zero_step picks (mirrors the library's rule)
     tma_path = (not args.two_pass and w["stage"] != 3 and not args.no_tma and
-                (args.tma or (w["Nd"] >= 16 and (w["bucket"] or w["N"]) >= (1 << 26))))
+                (args.tma or (w["Nd"] >= 16 and (w["bucket"] or w["N"]) >= (1 << 24))))
     if w["stage"] == 3 and args.fused_layers:
         line_kernel = "zero3 step: gather_layer + fused_step kernels (per layer)"
     elif w["stage"] == 3:

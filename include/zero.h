@@ -249,7 +249,7 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
  *     (bucket = 0: one bucket).  Two kernels implement the pass with identical results: a
  *     register-pipelined one (16-byte vector loads and stores) and a TMA-pipelined one (bulk
  *     copies through a shared-memory ring, bulk-store fan-out to the replicas).  The TMA one is
- *     chosen for wide fan-in (Nd >= 16) over buckets of at least 2^26 elements when every buffer
+ *     chosen for wide fan-in (Nd >= 16) over buckets of at least 2^24 elements when every buffer
  *     is 16-byte aligned; ZERO_NO_TMA / ZERO_FORCE_TMA in flags override the choice.  The pass reads state copy `live` and writes copy 1-live and
  *     the Nd weight replicas; when the step ends without overflow the copies swap, otherwise
  *     the replicas are rewritten from the unchanged state.  Stages 1 and 2 compute the same

@@ -289,7 +289,7 @@ int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s, bool depende
 
 // TMA-pipelined fused step over [a.lo, a.hi): whole tiles through the bulk-copy pipeline, the
 // rest by the same kernel's consumers.  Every pointer must be 16-byte aligned.
-int launch_fused_tma(int dtype, zb::TmaArgs& a, cudaStream_t s) {
+int launch_fused_tma(int dtype, zb::TmaArgs& a, cudaStream_t s, bool dependent = false) {
   int sms = 0;
   int rc = tma_setup(&sms);
   if (rc) return rc;
@@ -309,10 +309,21 @@ int launch_fused_tma(int dtype, zb::TmaArgs& a, cudaStream_t s) {
   if (grid < 1) grid = 1;
   a.stall_unit = g_test_stall;
   g_test_stall = -1;
-  if (dtype == ZERO_FP16)
-    zb::fused_step_tma_kernel<1><<<(unsigned)grid, zb::kTmaThreads, zb::kTmaSmemBytes, s>>>(a);
-  else
-    zb::fused_step_tma_kernel<0><<<(unsigned)grid, zb::kTmaThreads, zb::kTmaSmemBytes, s>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(zb::kTmaThreads);
+  cfg.dynamicSmemBytes = zb::kTmaSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (dependent) {  // a later bucket of the same step: may overlap the previous bucket's tail
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  const cudaError_t e = dtype == ZERO_FP16 ? cudaLaunchKernelEx(&cfg, zb::fused_step_tma_kernel<1>, a)
+                                           : cudaLaunchKernelEx(&cfg, zb::fused_step_tma_kernel<0>, a);
+  if (e != cudaSuccess) return cuda_fail(e, "fused_step_tma_kernel launch");
   return check_launch("fused_step_tma_kernel launch");
 }
 
@@ -888,11 +899,12 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   a.Nd = Nd;
   a.nrep = Nd;
   a.vec = al;
-  // The TMA pipeline wins where many loads must be in flight per element over a long window
-  // (same box, with its multi-wave grid: Nd = 64, 2^28: 6671 GB/s against 6091 for the register
-  // kernel; Nd = 16, 1.3e9 in one bucket: 6635 against 6229); at Nd = 8 the two are equal, and
-  // a TMA launch has a fixed cost (~22 us) that hurts short bucketed windows.
-  const bool tma_auto = Nd >= 16 && B >= (int64_t(1) << 26);
+  // The TMA pipeline wins where many loads must be in flight per element (same box, with its
+  // multi-wave grid: Nd = 64, 2^28: 6671 GB/s against 6091 for the register kernel; Nd = 16,
+  // 1.3e9 in one bucket: 6635 against 6229; in 52 buckets of 25M, with the buckets launched as
+  // programmatic dependents, which hides the TMA kernel's per-launch set-up: 6555 against 6115);
+  // at Nd = 8 the two are equal.  Windows under 2^24 elements keep the register kernel.
+  const bool tma_auto = Nd >= 16 && B >= (int64_t(1) << 24);
   const bool tma = al && !(st->flags & ZERO_NO_TMA) && ((st->flags & ZERO_FORCE_TMA) || tma_auto);
   zb::TmaArgs ta;
   if (tma) {
@@ -920,7 +932,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       ta.lo = a.lo;
       ta.hi = a.hi;
       ta.mode = a.mode;
-      if ((rc = launch_fused_tma(st->grad_dtype, ta, s))) return rc;
+      if ((rc = launch_fused_tma(st->grad_dtype, ta, s, k > 0))) return rc;
     } else if ((rc = launch_fused(st->grad_dtype, a, s, k > 0))) {
       return rc;
     }

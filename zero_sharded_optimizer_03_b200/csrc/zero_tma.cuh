@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_launch_dependents();  // a later bucket may take each SM as soon as this CTA leaves it
   const Bias b = s_bias;
   const int live = s_live;
   const float inv = s_inv;
@@ -373,6 +374,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
         wait_drain(full_bar((int)(u % kStages)), (uint32_t)((u / kStages) & 1));
     }
   }
+  pdl_wait();  // a programmatic dependent: the previous bucket has completed
   block_finish<kTmaWarps>(sq, bad, a.hdr, a.part, a.mode);
 }
 
