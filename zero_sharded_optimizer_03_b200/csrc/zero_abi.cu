@@ -116,6 +116,7 @@ int grid_for(int kid, int64_t work, int* grid, int waves = 1, bool partials = tr
 constexpr int kWavesRs = 4;
 constexpr int kWavesAdam = 8;
 constexpr int kWavesGather = 16;
+constexpr int kWavesGatherTma = 32;
 
 // Fused kernel over a long window: chunks handed out by the workspace counter, or the fixed
 // grid-stride split.  Same-box sweeps at 2^25-2^28 elements, chunks against the best fixed grid:
@@ -427,7 +428,9 @@ int do_gather_tma(const uint16_t* const* shards, int Nd, int64_t L, uint16_t* co
   a.S = S;
   a.hdr = header(ws);
   const int64_t chunks = (S + zb::kGTile - 1) / zb::kGTile;
-  int64_t gx = ((int64_t)sms * gather_tma_per_sm() + Nd - 1) / Nd;  // about one wave over the Nd rows
+  // about kWavesGatherTma waves over the Nd rows (same-box sweep on a 202M-element layer, Nd = 8:
+  // 1 wave 5708 GB/s, 8 waves 6335, 32 waves 6570; the register gather with 16 waves 5979)
+  int64_t gx = ((int64_t)sms * gather_tma_per_sm() * kWavesGatherTma + Nd - 1) / Nd;
   if (gx > chunks) gx = chunks;
   if (gx < 1) gx = 1;
   zb::gather_layer_tma_kernel<<<dim3((unsigned)gx, Nd), 32, zb::kGSmemBytes, s>>>(a);
@@ -752,8 +755,9 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
         outs[r] = st->params[r] + l * st->param_layer_stride;
         gl[r] = st->grads[r] + l * st->grad_layer_stride;
       }
-      // register gather by default (16 waves: 5.98 TB/s against 5.35 for the TMA fan-out on
-      // the 202M-element layer); ZERO_FORCE_TMA selects the TMA version
+      // register gather by default; ZERO_FORCE_TMA selects the TMA fan-out.  Alone on a
+      // 202M-element layer the TMA one is faster (32 waves: 6.57 TB/s against 5.98), but inside
+      // the ZeRO-3 step the two measured the same (69.16 against 68.93 ms per step)
       rc = (st->flags & ZERO_FORCE_TMA) ? do_gather_tma(shards, Nd, Ll, outs, Nd, ws, s)
                                         : do_gather(shards, Nd, Ll, outs, Nd, s);
       if (rc) return rc;
