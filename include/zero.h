@@ -277,7 +277,8 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t *
 /* Tracing hook.  Registers two cudaEvent_t handles (passed as void*) for the next zero_step
  * call on this thread: `start_event` is recorded on its stream just before the first kernel
  * that reads gradients and `stop_event` just after the last kernel that writes state (for
- * ZERO_FUSED: around the fused kernels, before the overflow-repair check).  One-shot: the
+ * ZERO_FUSED and ZERO_FUSED_LAYERS: the fused kernels and the overflow-repair check that
+ * follows them, which is a no-op unless the step overflowed).  One-shot: the
  * registration is cleared once each event is recorded.  NULL clears.  The events stay owned
  * by the caller.  Always returns ZERO_OK. */
 int zero_profile_events(void *start_event, void *stop_event);

@@ -357,11 +357,25 @@ int launch_adam(const zb::AdamArgs& a, cudaStream_t s) {
   return check_launch("adam_kernel launch");
 }
 
-int launch_cast(const zb::CastArgs& a, cudaStream_t s) {
+// dependent: the overflow repair right after the step's last fused launch on the same stream
+// (programmatic dependent launch: its launch overlaps the fused kernel's tail).
+int launch_cast(const zb::CastArgs& a, cudaStream_t s, bool dependent = false) {
   int grid = 0;
   int rc = grid_for(kCast, (a.hi - a.lo + 7) / 8, &grid);
   if (rc) return rc;
-  zb::cast_allgather_kernel<<<grid, zb::kThreads, 0, s>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(zb::kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (dependent) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, zb::cast_allgather_kernel, a);
+  if (e != cudaSuccess) return cuda_fail(e, "cast_allgather_kernel launch");
   return check_launch("cast_allgather_kernel launch");
 }
 
@@ -513,12 +527,13 @@ static int zero3_fused_layers(int Nd, int64_t N, int64_t bucket, const zero_stat
     a.Nd = Nd;
     a.vec = fal;
     a.mode = (l == 0 ? zb::kAccSet : zb::kAccAdd) | (l == nl - 1 ? (zb::kFinalize | zb::kFlip) : 0);
+    a.trigger_late = l == nl - 1;  // followed by the repair check
     if ((rc = launch_fused(st->grad_dtype, a, s))) return rc;
     off += Sl * Nd;
   }
-  prof_mark(false, s);
   // overflow repair: the bf16 shards from the unchanged live copy (runs only after a skip); the
-  // shards and the state share one padded layout, so one launch covers every layer
+  // shards and the state share one padded layout, so one launch covers every layer.  Launched
+  // as a programmatic dependent of the last fused launch, inside the traced span.
   zb::CastArgs r;
   std::memset(&r, 0, sizeof r);
   r.src[0] = st->master[0];
@@ -530,7 +545,9 @@ static int zero3_fused_layers(int Nd, int64_t N, int64_t bucket, const zero_stat
   r.hi = off;
   r.hdr = header(ws);
   r.vec = aligned16(r.src[0]) && aligned16(r.src[1]) && aligned16(r.reps[0]);
-  return launch_cast(r, s);
+  rc = launch_cast(r, s, true);
+  prof_mark(false, s);
+  return rc;
 }
 
 // ==================================================================== C ABI
@@ -932,17 +949,19 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     a.lo = k * B < N ? k * B : N;
     a.hi = (k + 1) * B < N ? (k + 1) * B : N;
     a.mode = (k == 0 ? zb::kAccSet : zb::kAccAdd) | (k == nb - 1 ? (zb::kFinalize | zb::kFlip) : 0);
+    a.trigger_late = k == nb - 1;  // followed by the repair check, not by another bucket
     if (tma) {
       ta.lo = a.lo;
       ta.hi = a.hi;
       ta.mode = a.mode;
+      ta.trigger_late = a.trigger_late;
       if ((rc = launch_fused_tma(st->grad_dtype, ta, s, k > 0))) return rc;
     } else if ((rc = launch_fused(st->grad_dtype, a, s, k > 0))) {
       return rc;
     }
   }
-  prof_mark(false, s);
-  // overflow repair: rewrite the replicas from the unchanged state (runs only after a skip)
+  // overflow repair: rewrite the replicas from the unchanged state (runs only after a skip);
+  // launched as a programmatic dependent of the last fused launch, inside the traced span
   zb::CastArgs r;
   std::memset(&r, 0, sizeof r);
   r.src[0] = st->master[0];
@@ -954,7 +973,9 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   r.hi = N;
   r.hdr = header(ws);
   r.vec = al;
-  return launch_cast(r, s);
+  rc = launch_cast(r, s, true);
+  prof_mark(false, s);
+  return rc;
 }
 
 }  // extern "C"

@@ -367,7 +367,7 @@ struct FusedArgs {
   int vec;
   int nrep;     // bf16 outputs per element: the Nd replicas (ZeRO-1/2), or 1 (a ZeRO-3 layer's shard)
   int chunked;  // 1: CTAs take chunks of kChunkVecs vectors from hdr->chunk (needs mode != 0)
-  int unused;
+  int trigger_late;  // 1: a dependent launch may start only once this CTA's main loop is done
 };
 
 // Programmatic dependent launch: a grid launched with programmatic stream serialization may
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
     s_live = __ldcg(&a.hdr->live) & 1;
     s_inv = step_inv(a.c, a.hdr);
   }
-  pdl_launch_dependents();
+  if (!a.trigger_late) pdl_launch_dependents();  // the next bucket may fill this launch's tail
   __syncthreads();
   const Bias b = s_bias;
   const int live = s_live;
@@ -469,6 +469,9 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
 #pragma unroll 1
     for (int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x; j < sp8.nvec; j += stride) vector_step(j);
   }
+  // before a dependent that only waits for this grid (the overflow-repair check), trigger late:
+  // its CTAs would otherwise sit on the SMs for the whole of this launch
+  if (a.trigger_late) pdl_launch_dependents();
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
     const int64_t i = sp8.scalar_index(a.lo, e);
@@ -661,8 +664,11 @@ struct CastArgs {
   int unused;
 };
 
+// The overflow repair after a fused step may be launched as a programmatic dependent of the last
+// fused launch: it waits for that grid (its header and replica writes) before anything else.
 __global__ void __launch_bounds__(kThreads) cast_allgather_kernel(const __grid_constant__ CastArgs a) {
   __shared__ int s_run, s_live;
+  pdl_wait();
   if (threadIdx.x == 0) {
     int run = 1, live = 0;
     if (a.gate == kGateNoOverflow) run = !__ldcg(&a.hdr->pending_flag);

@@ -172,6 +172,8 @@ struct TmaArgs {
   Partial* part;
   int Nd;
   int mode;
+  int trigger_late;    // 1: a dependent launch may start only once this CTA's tiles are done
+  int unused;
   int64_t stall_unit;  // test hook: CTA 0 issues no copies for this load unit (-1: none)
 };
 
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
     fence_barrier_init();
   }
   __syncthreads();
-  pdl_launch_dependents();  // a later bucket may take each SM as soon as this CTA leaves it
+  if (!a.trigger_late) pdl_launch_dependents();  // a later bucket may take each SM as soon as this CTA leaves it
   const Bias b = s_bias;
   const int live = s_live;
   const float inv = s_inv;
@@ -374,6 +376,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) fused_step_tma_kernel(const __
         wait_drain(full_bar((int)(u % kStages)), (uint32_t)((u / kStages) & 1));
     }
   }
+  if (a.trigger_late) pdl_launch_dependents();
   pdl_wait();  // a programmatic dependent: the previous bucket has completed
   block_finish<kTmaWarps>(sq, bad, a.hdr, a.part, a.mode);
 }
