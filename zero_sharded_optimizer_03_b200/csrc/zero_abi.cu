@@ -75,9 +75,9 @@ std::mutex g_dev_mu;
 // of resident CTAs (`waves` x SMs x CTAs per SM).  Several waves let the block scheduler hand
 // the later CTAs to whichever SMs finish first, instead of every SM owning a fixed 1/148 of the
 // data; measured on B200 (same-box sweeps of 1, 2, 4, 8 and 16 waves), that balancing is worth
-// up to 20% for the in-place Adam kernel and 12% for the layer gather, and nothing or a little
-// less for the fused kernel at 2 or 8 replicas per batch.  Kernels that leave a per-CTA partial
-// in the workspace are capped at kMaxCtas CTAs.
+// up to 20% for the in-place Adam kernel and 12% for the layer gather.  (The register fused
+// kernel keeps one wave and balances with chunks instead, see use_chunks.)  Kernels that leave
+// a per-CTA partial in the workspace are capped at kMaxCtas CTAs.
 int grid_for(int kid, int64_t work, int* grid, int waves = 1, bool partials = true) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
