@@ -1,0 +1,88 @@
+"""The oracle's pins catch plausible mistakes: each case plants one slip in a scratch copy of the
+oracle's C source (a dropped term, a wrong constant, operand or index, a reversed order, floor
+instead of ceiling, a different rounding rule), rebuilds that copy and runs the pins against it
+(tests/test_oracle_pins.py, on the CPU).  Every planted slip must fail at least one pin.  The
+repository's oracle is never modified; the copies live in a temporary directory.
+
+Left out on purpose: letting the Adam loop also update a shard's zero padding (returning the
+padded shard length) is an equivalent change -- padding has zero gradient and zero state, which
+the update maps to zero -- so no pin can or should catch it."""
+import os
+import shutil
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# (what the slip is, exact text in oracle/zero_oracle.c, planted text)
+MUTATIONS = [
+    ("eps inside the bias-corrected denominator",
+     "float den = sqrtf(vi) / c->sbc2 + c->eps;", "float den = (sqrtf(vi) + c->eps) / c->sbc2;"),
+    ("decoupled weight decay dropped",
+     "if (c->apply_decay) pi = pi * c->decay;", "(void)0;"),
+    ("beta2 used in the first-moment update",
+     "float mi = c->beta1 * m[i] + c->omb1 * g[i];", "float mi = c->beta2 * m[i] + c->omb1 * g[i];"),
+    ("replicas summed in reverse rank order",
+     "for (int q = 0; q < Nd; q++) s = s + grad_value(grads[q], i, dtype);",
+     "for (int q = Nd - 1; q >= 0; q--) s = s + grad_value(grads[q], i, dtype);"),
+    ("shard length rounded down",
+     "if (S * Nd < N) S = S + 1;", "(void)0;"),
+    ("bf16 rounding ties away from zero",
+     "if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) kept = kept + 1u;",
+     "if (dropped >= 0x8000u) kept = kept + 1u;"),
+    ("first-moment bias correction missing",
+     "c->step_size = (float)(lr / bc1);", "c->step_size = (float)lr;"),
+    ("square root of the second-moment correction missing",
+     "c->sbc2 = (float)sqrt(bc2);", "c->sbc2 = (float)bc2;"),
+    ("gradient summed, not averaged over ranks",
+     "double denom = average ? (double)Nd * ls : ls;", "double denom = ls;"),
+    ("overflow check removed",
+     "if (!isfinite(g)) *overflow = 1;", "(void)0;"),
+    ("fp16 exponent bias off by one",
+     "mag = ldexp((double)(1024 + frac), e - 25);", "mag = ldexp((double)(1024 + frac), e - 24);"),
+    ("layer gather reads the wrong shard element",
+     "if (j < L) full[j] = shards[r][k];", "if (j < L) full[j] = shards[r][k ? k - 1 : 0];"),
+    ("second-moment update loses a factor of g",
+     "float vi = c->beta2 * v[i] + (c->omb2 * g[i]) * g[i];",
+     "float vi = c->beta2 * v[i] + c->omb2 * g[i];"),
+]
+
+
+def _run_mutant(k, old, new, base):
+    d = os.path.join(base, "m%s" % k)
+    os.makedirs(d)
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(d, "oracle"),
+                    ignore=shutil.ignore_patterns("*.so", "*.tmp.*", "__pycache__"))
+    shutil.copytree(os.path.join(ROOT, "synth"), os.path.join(d, "synth"),
+                    ignore=shutil.ignore_patterns("__pycache__"))
+    shutil.copy(os.path.join(ROOT, "tests", "test_oracle_pins.py"), d)
+    src = os.path.join(d, "oracle", "zero_oracle.c")
+    text = open(src).read()
+    if old is not None:  # None: the unmodified control copy
+        assert text.count(old) >= 1, "mutation %d does not apply: %r" % (k, old)
+        open(src, "w").write(text.replace(old, new))  # every occurrence (e.g. each reduce loop)
+    env = dict(os.environ)
+    env.pop("PYTHONPATH", None)
+    p = subprocess.run([sys.executable, "-m", "pytest", "--noconftest", "-p", "no:cacheprovider",
+                        "-x", "-q", "test_oracle_pins.py"], cwd=d, env=env, capture_output=True,
+                       text=True, timeout=900)
+    return p.returncode, p.stdout[-2000:]
+
+
+def test_every_planted_slip_fails_a_pin(tmp_path):
+    with ThreadPoolExecutor(max_workers=min(len(MUTATIONS) + 1, os.cpu_count() or 4)) as ex:
+        control = ex.submit(_run_mutant, "control", None, None, str(tmp_path))
+        futs = [ex.submit(_run_mutant, k, old, new, str(tmp_path))
+                for k, (_, old, new) in enumerate(MUTATIONS)]
+        results = [f.result() for f in futs]
+        rc, out = control.result()
+    # the unmodified copy passes the same pins the same way, so a failure below is the slip's
+    assert rc == 0, "unmodified oracle copy fails its pins (exit %d)\n%s" % (rc, out)
+    survivors = []
+    for (what, _, _), (rc, out) in zip(MUTATIONS, results):
+        # pytest exit code 1: some pin failed (the planted slip was caught); anything else --
+        # 0 (all passed) or 2-5 (the run itself broke) -- is not a catch
+        if rc != 1:
+            survivors.append("%s (pytest exit %d)\n%s" % (what, rc, out))
+    assert not survivors, "\n\n".join(survivors)
