@@ -1,7 +1,8 @@
 """The oracle's pins catch plausible mistakes: each case plants one slip in a scratch copy of the
 oracle's C source (a dropped term, a wrong constant, operand or index, a reversed order, floor
 instead of ceiling, a different rounding rule), rebuilds that copy and runs the pins against it
-(tests/test_oracle_pins.py, on the CPU).  Every planted slip must fail at least one pin.  The
+(tests/test_oracle_pins.py, test_oracle_scaler_clip.py and test_oracle_accounting.py, on the
+CPU).  Every planted slip must fail at least one pin.  The
 repository's oracle is never modified; the copies live in a temporary directory.
 
 Left out on purpose: letting the Adam loop also update a shard's zero padding (returning the
@@ -46,7 +47,29 @@ MUTATIONS = [
     ("second-moment update loses a factor of g",
      "float vi = c->beta2 * v[i] + (c->omb2 * g[i]) * g[i];",
      "float vi = c->beta2 * v[i] + c->omb2 * g[i];"),
+    # dynamic loss scale, clipping, the bf16-kept reduced gradient
+    ("loss scale grows instead of backing off after an overflow",
+     "*scale = *scale * backoff;", "*scale = *scale * growth;"),
+    ("loss scale grows one clean step late",
+     "if (*good >= interval) {", "if (*good > interval) {"),
+    ("loss scale may leave the finite fp32 range",
+     "if (grown <= fp32_max) *scale = grown;", "*scale = grown;"),
+    ("clipping by the sum of squares instead of the norm",
+     "double coef = max_norm / (sqrt(sumsq) + 1e-6);", "double coef = max_norm / (sumsq + 1e-6);"),
+    ("clipping factor allowed above 1",
+     "if (coef > 1.0) coef = 1.0;", "(void)0;"),
+    ("bf16-kept gradient not rounded",
+     "float g = oracle_bf16_to_f32(oracle_f32_to_bf16(s * inv));", "float g = s * inv;"),
+    # memory and communication accounting
+    ("ZeRO-1 counted as partitioning the gradients",
+     "double g[4] = {G, G, G / d, G / d};", "double g[4] = {G, G / d, G / d, G / d};"),
+    ("ZeRO-3 communication counted like ZeRO-1/2",
+     "if (stage == 3) return 3.0 * one;", "if (stage == 3) return 2.0 * one;"),
+    ("ring collective volume without the (Nd-1)/Nd factor",
+     "double one = (double)(Nd - 1) / (double)Nd * N;", "double one = N;"),
 ]
+
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_scaler_clip.py", "test_oracle_accounting.py"]
 
 
 def _run_mutant(k, old, new, base):
@@ -56,7 +79,9 @@ def _run_mutant(k, old, new, base):
                     ignore=shutil.ignore_patterns("*.so", "*.tmp.*", "__pycache__"))
     shutil.copytree(os.path.join(ROOT, "synth"), os.path.join(d, "synth"),
                     ignore=shutil.ignore_patterns("__pycache__"))
-    shutil.copy(os.path.join(ROOT, "tests", "test_oracle_pins.py"), d)
+    for f in PIN_FILES:
+        shutil.copy(os.path.join(ROOT, "tests", f), d)
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(d, "golden"))
     src = os.path.join(d, "oracle", "zero_oracle.c")
     text = open(src).read()
     if old is not None:  # None: the unmodified control copy
@@ -65,7 +90,7 @@ def _run_mutant(k, old, new, base):
     env = dict(os.environ)
     env.pop("PYTHONPATH", None)
     p = subprocess.run([sys.executable, "-m", "pytest", "--noconftest", "-p", "no:cacheprovider",
-                        "-x", "-q", "test_oracle_pins.py"], cwd=d, env=env, capture_output=True,
+                        "-x", "-q", *PIN_FILES], cwd=d, env=env, capture_output=True,
                        text=True, timeout=900)
     return p.returncode, p.stdout[-2000:]
 
