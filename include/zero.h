@@ -250,10 +250,15 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
  *     register-pipelined one (16-byte vector loads and stores) and a TMA-pipelined one (bulk
  *     copies through a shared-memory ring, bulk-store fan-out to the replicas).  The TMA one is
  *     chosen for wide fan-in (Nd >= 16) over buckets of at least 2^24 elements when every buffer
- *     is 16-byte aligned; ZERO_NO_TMA / ZERO_FORCE_TMA in flags override the choice.  The pass reads state copy `live` and writes copy 1-live and
- *     the Nd weight replicas; when the step ends without overflow the copies swap, otherwise
- *     the replicas are rewritten from the unchanged state.  Stages 1 and 2 compute the same
- *     values (they differ in what a real cluster keeps in memory, see zero_memory_estimate).
+ *     is 16-byte aligned; ZERO_NO_TMA / ZERO_FORCE_TMA in flags override the choice.  The pass
+ *     reads state copy `live` and writes copy 1-live and the Nd weight replicas; when the step
+ *     ends without overflow the copies swap, otherwise the replicas are rewritten from the
+ *     unchanged state.  Stages 1 and 2 compute the same values (they differ in what a real
+ *     cluster keeps in memory, see zero_memory_estimate).  Buckets after the first, and the
+ *     overflow-repair check after the last, are programmatic dependent launches on `stream`
+ *     (each may start while the previous kernel of the step finishes; it waits for that kernel
+ *     before using its results), so nothing else should be enqueued between them: one
+ *     zero_step call enqueues the whole step.
  *   stage 1/2, ZERO_TWO_PASS: reduce-scatter into grad_shard, then (if no overflow) Adam in
  *     place on copy 0 fused with the cast and the all-gather.
  *   stage 3: N elements in layers of `bucket` elements (the last may be shorter; bucket = 0
