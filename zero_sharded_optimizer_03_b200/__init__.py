@@ -302,7 +302,9 @@ class ZeroBuffers:
     an fp32 gradient shard (ZERO_TWO_PASS).
     stage 3: `layers` layers of `layer_len` elements (the last may be shorter), every layer
     padded to a multiple of Nd; one layer-sized gradient buffer and one gathered-weight
-    buffer per rank (reused for every layer unless per_layer_buffers is set).
+    buffer per rank (reused for every layer unless per_layer_buffers is set); one fp32 state
+    copy and a reduced-gradient shard, or, with ZERO_FUSED_LAYERS, two state copies and no
+    gradient shard.
     """
 
     def __init__(self, stage: int, Nd: int, N: int, grad_dtype: int = ZERO_BF16,
