@@ -43,6 +43,47 @@ def test_every_declared_symbol_is_exported(zero):
         assert getattr(lib, n) is not None
 
 
+def test_binding_constants_match_the_header(zero):
+    """Every integer #define of include/zero.h has the same value in the Python binding."""
+    text = open(os.path.join(ROOT, "include", "zero.h")).read()
+    defines = dict(re.findall(r"#define\s+(ZERO_[A-Z0-9_]+)\s+\(?(-?\d+)\)?\s", text))
+    assert len(defines) >= 15
+    for name, value in defines.items():
+        assert getattr(zero, name) == int(value), name
+    assert zero.ZERO_NOALLOC_MAX_WINDOW == zero.ZERO_NOALLOC_MAX_CTAS * 2048
+
+
+STRUCTS = ["zero_partition_t", "zero_hparams_t", "zero_step_result_t", "zero_state_t",
+           "zero_mem_t", "zero_rs_summary_t", "zero_offload_state_t"]
+
+
+def test_binding_structures_match_the_header_layout(zero, tmp_path):
+    """The ctypes structures have the size and field offsets that a C compiler gives the
+    header's structures (compiled here with gcc against include/zero.h)."""
+    fields = {n: [f[0] for f in getattr(zero, n)._fields_] for n in STRUCTS}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "zero.h"', "int main(void) {"]
+    for n in STRUCTS:
+        lines.append('printf("%s size %%zu\\n", sizeof(%s));' % (n, n))
+        for f in fields[n]:
+            lines.append('printf("%s %s %%zu\\n", offsetof(%s, %s));' % (n, f, n, f))
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    want = {}
+    for line in out.splitlines():
+        n, f, v = line.split()
+        want[(n, f)] = int(v)
+    for n in STRUCTS:
+        cls = getattr(zero, n)
+        assert ctypes.sizeof(cls) == want[(n, "size")], n
+        for f in fields[n]:
+            assert getattr(cls, f).offset == want[(n, f)], (n, f)
+
+
 def test_partition_matches_oracle(zero):
     for Nd in (1, 2, 3, 4, 7, 8, 16, 64):
         for N in list(range(0, 70)) + [1_000_003, 124_439_808, 6_476_005_376]:
