@@ -212,3 +212,27 @@ def test_offload_step_validates_before_touching_the_device(zero):
     with pytest.raises(zero.ZeroError) as e:
         zero.zero_offload_step(4, 10, 0, st, hp)
     assert "grad_dev" in str(e.value)
+
+
+def test_workspace_header_offsets_used_by_the_multi_gpu_path(tmp_path):
+    """dist.py all-reduces the pending overflow flag and sum of squares in place in the
+    workspace header by byte offset; the device header (compiled here for the host with nvcc,
+    nothing runs on a GPU) has them at those offsets, fits its 256-byte slot, and is what
+    zero_read_result copies."""
+    from zero_sharded_optimizer_03_b200 import dist
+    src = tmp_path / "hdr.cu"
+    src.write_text(
+        '#include <cstdio>\n#include <cstddef>\n#include "zero_kernels.cuh"\n'
+        "int main() {\n"
+        '  std::printf("%zu %zu %zu\\n", offsetof(zb::Header, pending_flag),\n'
+        "              offsetof(zb::Header, pending_sumsq), sizeof(zb::Header));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "hdr"
+    nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    subprocess.run([nvcc, "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-I",
+                    os.path.join(ROOT, "zero_sharded_optimizer_03_b200", "csrc"), str(src),
+                    "-o", str(exe)], check=True)
+    flag, sumsq, size = map(int, subprocess.run([str(exe)], capture_output=True, text=True,
+                                                check=True).stdout.split())
+    assert (flag, sumsq) == (dist.PENDING_FLAG_OFFSET, dist.PENDING_SUMSQ_OFFSET)
+    assert size <= 256
