@@ -60,6 +60,18 @@ MUTATIONS = [
      "if (coef > 1.0) coef = 1.0;", "(void)0;"),
     ("bf16-kept gradient not rounded",
      "float g = oracle_bf16_to_f32(oracle_f32_to_bf16(s * inv));", "float g = s * inv;"),
+    # the all-gather and the per-element driver used for full-size sampled checks
+    ("all-gather skips the last replica",
+     "    for (int dst = 0; dst < Nd; dst++)\n        for (int r = 0; r < Nd; r++)",
+     "    for (int dst = 0; dst < Nd - 1; dst++)\n        for (int r = 0; r < Nd; r++)"),
+    ("sampled elements read the gradient matrix transposed",
+     "for (int q = 0; q < Nd; q++) s = s + grad_value(grads, e * Nd + q, dtype);\n        float g = s * c.inv;\n        if (gout)",
+     "for (int q = 0; q < Nd; q++) s = s + grad_value(grads, q * n + e, dtype);\n        float g = s * c.inv;\n        if (gout)"),
+    ("sampled elements updated on a skipped step",
+     "if (!skip) oracle_adam(p + e, m + e, v + e, &g, 1, &c);", "oracle_adam(p + e, m + e, v + e, &g, 1, &c);"),
+    ("sampled elements of the clipping driver updated on a skipped step",
+     "float g = (s * c.inv) * coef;\n        if (!skip) oracle_adam(p + e, m + e, v + e, &g, 1, &c);",
+     "float g = (s * c.inv) * coef;\n        oracle_adam(p + e, m + e, v + e, &g, 1, &c);"),
     # memory and communication accounting
     ("ZeRO-1 counted as partitioning the gradients",
      "double g[4] = {G, G, G / d, G / d};", "double g[4] = {G, G / d, G / d, G / d};"),

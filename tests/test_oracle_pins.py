@@ -376,3 +376,31 @@ def test_update_elements_matches_full_step():
     g_en = np.stack(grads, axis=1)
     out16, _ = oracle.update_elements(Nd, oracle.BF16, g_en, p_e, m_e, v_e, HP, t, skip=False)
     assert p_e.tobytes() == master[:N].tobytes() and (out16 == reps[0]).all()
+
+
+def test_update_elements_on_a_skipped_step_change_nothing():
+    """A skipped step (an overflow anywhere) leaves the sampled elements' state as it was and
+    reports the unchanged weights, as the full step does."""
+    Nd, N = 3, 29
+    S, Np, _ = oracle.partition(N, Nd)
+    master, m, v = _state(N, Np)
+    grads = _rand_grads(Nd, N, oracle.BF16)
+    p0, m0, v0 = master[:N].copy(), m[:N].copy(), v[:N].copy()
+    p_e, m_e, v_e = p0.copy(), m0.copy(), v0.copy()
+    out16, g = oracle.update_elements(Nd, oracle.BF16, np.stack(grads, axis=1), p_e, m_e, v_e, HP,
+                                      5, skip=True, want_grad=True)
+    assert (p_e.tobytes(), m_e.tobytes(), v_e.tobytes()) == (p0.tobytes(), m0.tobytes(),
+                                                             v0.tobytes())
+    assert (out16 == oracle.f32_to_bf16(p0)).all()
+    # the clipping variant of the per-element driver skips the same way
+    p_x, m_x, v_x = p0.copy(), m0.copy(), v0.copy()
+    out16x = oracle.update_elements_ex(Nd, oracle.BF16, np.stack(grads, axis=1), p_x, m_x, v_x,
+                                       HP, 5, True, np.float32(0.5))
+    assert (p_x.tobytes(), m_x.tobytes(), v_x.tobytes()) == (p0.tobytes(), m0.tobytes(),
+                                                             v0.tobytes())
+    assert (out16x == oracle.f32_to_bf16(p0)).all()
+    # the reduced gradient is still reported (rank-order mean), skip or not
+    want = np.zeros(N, np.float32)
+    for r in range(Nd):
+        want = want + oracle.bf16_to_f32(grads[r])
+    assert g.tobytes() == (want * np.float32(1.0 / Nd)).tobytes()
