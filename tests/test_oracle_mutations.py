@@ -72,6 +72,19 @@ MUTATIONS = [
     ("sampled elements of the clipping driver updated on a skipped step",
      "float g = (s * c.inv) * coef;\n        if (!skip) oracle_adam(p + e, m + e, v + e, &g, 1, &c);",
      "float g = (s * c.inv) * coef;\n        oracle_adam(p + e, m + e, v + e, &g, 1, &c);"),
+    # step bookkeeping, scalars, buckets, norms
+    ("bucket windows drop their last element",
+     "int64_t hi = lo + w < Np ? lo + w : Np;", "int64_t hi = lo + w - 1 < Np ? lo + w - 1 : Np;"),
+    ("weight decay factor without the learning rate",
+     "c->decay = (float)(1.0 - lr * wd);", "c->decay = (float)(1.0 - wd);"),
+    ("second-moment coefficient from beta1",
+     "c->omb2 = (float)(1.0 - b2);", "c->omb2 = (float)(1.0 - b1);"),
+    ("sum of squares accumulates g instead of g^2",
+     "*sumsq += (double)g * (double)g;", "*sumsq += (double)g;"),
+    ("unsharded reference forgets the unscale",
+     "g[i] = s * c.inv;\n        if (!isfinite(g[i])) *overflow = 1;", "g[i] = s;\n        if (!isfinite(g[i])) *overflow = 1;"),
+    ("clip factor computed but not applied",
+     "for (int64_t i = 0; i < N; i++) g[i] = g[i] * coef;", "(void)coef;"),
     # memory and communication accounting
     ("ZeRO-1 counted as partitioning the gradients",
      "double g[4] = {G, G, G / d, G / d};", "double g[4] = {G, G / d, G / d, G / d};"),
