@@ -1,6 +1,5 @@
 """The CPU half of ZeRO-Offload (zero_host_adam, product code that runs on the host) against the
 CPU oracle: bit-identical state and bf16 weights for any thread count, clipping factor and step."""
-import ctypes
 
 import numpy as np
 import pytest
