@@ -85,6 +85,12 @@ MUTATIONS = [
      "g[i] = s * c.inv;\n        if (!isfinite(g[i])) *overflow = 1;", "g[i] = s;\n        if (!isfinite(g[i])) *overflow = 1;"),
     ("clip factor computed but not applied",
      "for (int64_t i = 0; i < N; i++) g[i] = g[i] * coef;", "(void)coef;"),
+    # the ZeRO-3 layer layout
+    ("ZeRO-3 layers packed without their padding",
+     "        off += part[1];\n", "        off += layer_len[l];\n"),
+    ("ZeRO-3 bf16 shards not refreshed after the update",
+     "for (int64_t k = 0; k < n; k++) shard16[o + k] = oracle_f32_to_bf16(master[o + k]);",
+     "(void)n;"),
     # memory and communication accounting
     ("ZeRO-1 counted as partitioning the gradients",
      "double g[4] = {G, G, G / d, G / d};", "double g[4] = {G, G / d, G / d, G / d};"),
