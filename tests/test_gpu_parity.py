@@ -257,6 +257,30 @@ def test_long_windows_match_oracle(Nd, gdt, flags):
     free()
 
 
+@pytest.mark.parametrize("flags", [zero.ZERO_FUSED, zero.ZERO_TWO_PASS])
+def test_summed_gradient_option_matches_oracle(flags):
+    """grad_average = 0: the reduced gradient is the rank-order sum divided by the loss scale
+    only (no 1/Nd), on the fused and the two-pass paths; two steps, every element."""
+    Nd, N = 5, 30_011
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=4.0, grad_average=False)
+    buf = zero.ZeroBuffers(2, Nd, N, flags=flags)
+    _init_state(buf, N)
+    S, Np, _ = oracle.partition(N, Nd)
+    om, mm, vm = _host_state(N, Np)
+    oreps = [oracle.f32_to_bf16(om[:N]) for _ in range(Nd)]
+    t = 0
+    for step in (1, 2):
+        hg = [synth.fill_host(synth.NORMAL, synth.BF16, SEED, synth.grad_stream(step, r), N,
+                              sigma=4e-3) for r in range(Nd)]
+        for r in range(Nd):
+            fill(buf.grads[r], synth.NORMAL, synth.BF16, synth.grad_stream(step, r), sigma=4e-3)
+        buf.step(zero.hparams(**hp))
+        t, ovf, ss = oracle.zero12_step(Nd, N, 0, oracle.BF16, hg, om, mm, vm, oreps, hp, t)
+    _compare_full(buf, om, mm, vm, oreps, t, ss, "summed gradient")
+    del buf
+    free()
+
+
 def test_stage1_and_stage2_identical():
     Nd, N = 8, 300_001
     outs = []
