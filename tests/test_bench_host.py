@@ -75,3 +75,24 @@ def test_committed_traffic_records_are_consistent():
         assert abs(r["dram_bytes_per_launch"] - scaled) <= 1
         # DRAM traffic within a few percent of the algorithmic bytes (no re-reads)
         assert 0.9 <= r["dram_bytes_per_launch"] / r["algorithmic_bytes_per_launch"] <= 1.05
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the CPU oracle timed on the host) prints one JSON line with
+    the keys the benchmark contract asks of the reference arm."""
+    import subprocess
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                       timeout=600, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [x for x in p.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["unit"] == "params/s" and d["higher_is_better"] is True and d["value"] > 0
+    assert (d["steps"], d["warmup"], d["n_gpus"]) == (1, 3, 1)
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["config"]["workload"] == bench.WORKLOADS[bench.DEFAULT]["desc"]
