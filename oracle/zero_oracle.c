@@ -171,7 +171,7 @@ void oracle_reduce_scatter_window(int Nd, int64_t N, int dtype, const uint16_t *
                                   float inv, int64_t lo, int64_t hi, float *out,
                                   int *overflow, double *sumsq)
 {
-    int64_t part[3];
+    int64_t part[3] = {0, 0, 0};
     oracle_partition(N, Nd, part);
     int64_t S = part[0];
     for (int r = 0; r < Nd; r++) {
@@ -212,7 +212,7 @@ void oracle_adam(float *p, float *m, float *v, const float *g, int64_t n, const 
  * every rank's shard of the new weights, as bf16. */
 void oracle_allgather(int Nd, int64_t N, const float *master, uint16_t *const *replicas)
 {
-    int64_t part[3];
+    int64_t part[3] = {0, 0, 0};
     oracle_partition(N, Nd, part);
     int64_t S = part[0];
     for (int dst = 0; dst < Nd; dst++)
@@ -239,7 +239,7 @@ int oracle_zero12_step(int Nd, int64_t N, int64_t bucket, int dtype,
                        uint16_t *const *replicas, const double hp[7], int64_t *t,
                        int *overflow, double *sumsq)
 {
-    int64_t part[3];
+    int64_t part[3] = {0, 0, 0};
     if (oracle_partition(N, Nd, part) != 0 || bucket < 0) return -1;
     int64_t S = part[0], Np = part[1];
     float *g = (float *)malloc((size_t)(Np > 0 ? Np : 1) * sizeof(float));
@@ -306,7 +306,7 @@ int oracle_dp_step(int Nd, int64_t N, int dtype, const uint16_t *const *grads, f
  * rebuild the layer's L weights from its Nd shards of length S = ceil(L/Nd). */
 void oracle_zero3_gather(int Nd, int64_t L, const uint16_t *const *shards, uint16_t *full)
 {
-    int64_t part[3];
+    int64_t part[3] = {0, 0, 0};
     oracle_partition(L, Nd, part);
     int64_t S = part[0];
     for (int r = 0; r < Nd; r++)
@@ -331,7 +331,7 @@ int oracle_zero3_step(int Nd, int nlayers, const int64_t *layer_len, int dtype,
     if (Nd < 1 || nlayers < 0) return -1;
     int64_t total = 0;
     for (int l = 0; l < nlayers; l++) {
-        int64_t part[3];
+        int64_t part[3] = {0, 0, 0};
         if (oracle_partition(layer_len[l], Nd, part) != 0) return -1;
         total += part[1];
     }
@@ -348,7 +348,7 @@ int oracle_zero3_step(int Nd, int nlayers, const int64_t *layer_len, int dtype,
     *sumsq = 0.0;
     int64_t off = 0;
     for (int l = 0; l < nlayers; l++) {
-        int64_t part[3];
+        int64_t part[3] = {0, 0, 0};
         oracle_partition(layer_len[l], Nd, part);
         int64_t S = part[0];
         for (int r = 0; r < Nd; r++) sh[r] = shard16 + off + (int64_t)r * S;
@@ -368,7 +368,7 @@ int oracle_zero3_step(int Nd, int nlayers, const int64_t *layer_len, int dtype,
     oracle_scalars(hp, Nd, *t, &c);
     off = 0;
     for (int l = 0; l < nlayers; l++) {
-        int64_t part[3];
+        int64_t part[3] = {0, 0, 0};
         oracle_partition(layer_len[l], Nd, part);
         int64_t S = part[0];
         for (int r = 0; r < Nd; r++) {
@@ -507,7 +507,7 @@ void oracle_reduce_scatter_window_bf16(int Nd, int64_t N, int dtype, const uint1
                                        float inv, int64_t lo, int64_t hi, float *out, int *overflow,
                                        double *sumsq)
 {
-    int64_t part[3];
+    int64_t part[3] = {0, 0, 0};
     oracle_partition(N, Nd, part);
     int64_t S = part[0];
     for (int r = 0; r < Nd; r++) {
@@ -539,7 +539,7 @@ int oracle_zero12_step_ex(int Nd, int64_t N, int64_t bucket, int dtype, const ui
                           const double hpx[13], int64_t *t, double *scale, int64_t *good,
                           int *overflow, double *sumsq)
 {
-    int64_t part[3];
+    int64_t part[3] = {0, 0, 0};
     if (oracle_partition(N, Nd, part) != 0 || bucket < 0) return -1;
     int64_t S = part[0], Np = part[1];
     double hp[7];
