@@ -45,8 +45,15 @@ extern "C" {
 /* ------------------------------------------------------------------ codes and limits */
 
 #define ZERO_OK 0
-#define ZERO_EINVAL (-1) /* an argument is out of range or NULL; the message names it */
-#define ZERO_ECUDA (-2)  /* a CUDA runtime call or a kernel launch failed */
+#define ZERO_EINVAL (-1)   /* an argument is out of range or NULL; the message names it */
+#define ZERO_ECUDA (-2)    /* a CUDA runtime call or a kernel launch failed */
+#define ZERO_ENOMEM (-3)   /* the fixed scratch memory inside the library is too small for the
+                              request (zero_reduce_scatter_noalloc); caller-provided workspaces
+                              have a fixed size (zero_workspace_bytes) and cannot run short */
+#define ZERO_ETIMEOUT (-4) /* a kernel gave up a bounded internal wait (1 s).  Kernels run
+                              asynchronously, so this is recorded in the workspace error word
+                              when it happens and returned by the next synchronizing call,
+                              zero_read_result, which still fills its output */
 
 #define ZERO_MAX_ND 64   /* largest number of simulated data-parallel ranks */
 
@@ -186,7 +193,9 @@ int zero_workspace_init(void *ws, int64_t t, void *stream);
 int zero_loss_scaler_init(void *ws, double init_scale, double growth_factor, double backoff_factor,
                           int64_t growth_interval, void *stream);
 
-/* Copies the workspace bookkeeping to *out.  Synchronizes `stream` (waits for queued steps). */
+/* Copies the workspace bookkeeping to *out.  Synchronizes `stream` (waits for queued steps).
+ * Returns ZERO_ETIMEOUT, with *out filled, while the workspace error word is set (a bounded
+ * internal wait gave up in an earlier step; that step was skipped); ZERO_OK otherwise. */
 int zero_read_result(const void *ws, zero_step_result_t *out, void *stream);
 
 /* ------------------------------------------------------------------ building blocks */
@@ -312,7 +321,7 @@ typedef struct {
  * array inside the library: 256 B + 16 B x ZERO_NOALLOC_MAX_CTAS (about 256 KiB), held by every
  * GPU that loads the library until the process exits.  The call uses one CTA per 2048 elements,
  * so a window [lo, hi) may hold at most ZERO_NOALLOC_MAX_WINDOW elements; a larger window is
- * rejected with ZERO_EINVAL and a message naming the limit (split it into buckets).
+ * rejected with ZERO_ENOMEM and a message naming the limit (split it into buckets).
  *
  * grads, dtype, Nd, lo, hi, hp, grad_out: as for zero_reduce_scatter.  summary: device pointer the
  * call writes the window's result to (accumulate = 0), or combines it into (accumulate != 0:
@@ -414,7 +423,7 @@ int zero_offload_step(int Nd, int64_t N, int64_t chunk, const zero_offload_state
 /* Per-GPU model-state memory ([P1] §二 code: bytes_per_param for the 16-bit weights and again
  * for the gradients, bytes_per_opt_state for Adam's fp32 copy + m + v).  out[0] plain data
  * parallelism, out[1] ZeRO-1 (optimizer state / Nd), out[2] ZeRO-2 (also gradients / Nd),
- * out[3] ZeRO-3 (everything / Nd).  N >= 0, Nd >= 1. */
+ * out[3] ZeRO-3 (everything / Nd).  N >= 0, Nd >= 1, byte counts >= 0, else ZERO_EINVAL. */
 int zero_memory_estimate(double N, int Nd, int bytes_per_param, int bytes_per_opt_state,
                          zero_mem_t out[4]);
 

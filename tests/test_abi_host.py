@@ -114,6 +114,15 @@ def test_accounting_matches_oracle(zero):
     assert zero.zero_comm_volume(4, 1.0, 2) < 0 and zero.zero_comm_volume(1, 1.0, 0) < 0
 
 
+def test_accounting_rejections_leave_a_message(zero):
+    for args, word in [((-1.0, 4, 2, 12), "N"), ((1e9, 0, 2, 12), "Nd"),
+                       ((1e9, 4, -2, 12), "bytes_per_param")]:
+        zero.lib.zero_partition(-1, 4, None)  # leaves an unrelated message behind
+        with pytest.raises(zero.ZeroError) as e:
+            zero.zero_memory_estimate(*args)
+        assert e.value.code == zero.ZERO_EINVAL and word in str(e.value), args
+
+
 def test_workspace_and_version(zero):
     assert 256 < zero.zero_workspace_bytes() < (1 << 20)
     assert "sm_100a" in zero.zero_version()

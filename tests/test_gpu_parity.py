@@ -385,12 +385,17 @@ def test_bounded_wait_gives_up_reports_error_and_device_stays_usable():
     snap = [f32(buf.master[0]).tobytes()] + [u16(p).tobytes() for p in buf.params]
     zero.zero_test_inject_stall(2)  # CTA 0, tile 1, its gradient chunk
     buf.step(zero.hparams(**hp))
-    res = buf.result()
+    with pytest.raises(zero.ZeroTimeout) as e:  # the synchronizing read reports the timeout
+        buf.result()
+    assert e.value.code == zero.ZERO_ETIMEOUT
+    res = e.value.result
     assert res["error"] != 0 and res["overflow"] == 1 and res["skipped"] == 1 and res["step"] == 0
     assert res["live"] == 0
     assert [f32(buf.master[0]).tobytes()] + [u16(p).tobytes() for p in buf.params] == snap
     buf.step(zero.hparams(**hp))  # the hook was one-shot: this step commits
-    res = buf.result()
+    with pytest.raises(zero.ZeroTimeout) as e:  # the error word is sticky until init
+        buf.result()
+    res = e.value.result
     assert res["overflow"] == 0 and res["step"] == 1 and res["live"] == 1
     S, Np, _ = oracle.partition(N, Nd)
     om, mm, vm = _host_state(N, Np)

@@ -14,7 +14,7 @@ import ctypes
 import os
 
 __all__ = [
-    "ZeroError", "zero_partition", "zero_workspace_bytes", "zero_workspace_init",
+    "ZeroError", "ZeroTimeout", "zero_partition", "zero_workspace_bytes", "zero_workspace_init",
     "zero_read_result", "zero_begin_step", "zero_reduce_scatter", "zero_adam_shard",
     "zero_allgather", "zero_end_step", "zero3_gather_layer", "zero_step",
     "zero_memory_estimate", "zero_comm_volume", "zero_version", "zero_profile_events",
@@ -25,12 +25,13 @@ __all__ = [
     "LIB_PATH", "ZERO_BF16", "ZERO_FP16", "ZERO_FUSED", "ZERO_TWO_PASS", "ZERO_NO_TMA",
     "ZERO_FORCE_TMA", "ZERO_BF16_GRAD_SHARD", "ZERO_FUSED_LAYERS",
     "ZERO_GATE_ALWAYS",
-    "ZERO_GATE_NO_OVERFLOW", "ZERO_MAX_ND",
+    "ZERO_GATE_NO_OVERFLOW", "ZERO_MAX_ND", "ZERO_OK", "ZERO_EINVAL", "ZERO_ECUDA",
+    "ZERO_ENOMEM", "ZERO_ETIMEOUT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzero.so")
 
-ZERO_OK, ZERO_EINVAL, ZERO_ECUDA = 0, -1, -2
+ZERO_OK, ZERO_EINVAL, ZERO_ECUDA, ZERO_ENOMEM, ZERO_ETIMEOUT = 0, -1, -2, -3, -4
 ZERO_MAX_ND = 64
 ZERO_BF16, ZERO_FP16 = 0, 1
 ZERO_FUSED, ZERO_TWO_PASS, ZERO_NO_TMA, ZERO_FORCE_TMA, ZERO_BF16_GRAD_SHARD = 0, 1, 2, 4, 8
@@ -148,6 +149,15 @@ class ZeroError(RuntimeError):
         self.code = code
 
 
+class ZeroTimeout(ZeroError):
+    """ZERO_ETIMEOUT from zero_read_result: a kernel gave up a bounded wait in an earlier step
+    (that step was skipped).  `result` holds the bookkeeping the call still filled in."""
+
+    def __init__(self, code: int, msg: str, result: dict):
+        super().__init__(code, msg)
+        self.result = result
+
+
 def _check(rc: int) -> None:
     if rc != ZERO_OK:
         raise ZeroError(rc, lib.zero_last_error().decode())
@@ -187,10 +197,16 @@ def zero_workspace_init(ws: int, t: int = 0, stream: int = 0) -> None:
 
 
 def zero_read_result(ws: int, stream: int = 0) -> dict:
+    """The workspace bookkeeping as a dict.  Raises ZeroTimeout (carrying the dict) while the
+    workspace error word is set."""
     out = zero_step_result_t()
-    _check(lib.zero_read_result(ws, ctypes.byref(out), stream))
-    return {k: getattr(out, k) for k, _ in zero_step_result_t._fields_
-            if not k.startswith("reserved")}
+    rc = lib.zero_read_result(ws, ctypes.byref(out), stream)
+    res = {k: getattr(out, k) for k, _ in zero_step_result_t._fields_
+           if not k.startswith("reserved")}
+    if rc == ZERO_ETIMEOUT:
+        raise ZeroTimeout(rc, lib.zero_last_error().decode(), res)
+    _check(rc)
+    return res
 
 
 def zero_begin_step(ws: int, stream: int = 0) -> None:

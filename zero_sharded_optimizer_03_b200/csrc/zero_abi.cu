@@ -602,6 +602,11 @@ int zero_read_result(const void* ws, zero_step_result_t* out, void* stream) {
   out->good_steps = h.dyn ? h.good : 0;
   out->dynamic_scale = h.dyn;
   out->reserved3 = 0;
+  if (h.error)
+    return fail(ZERO_ETIMEOUT,
+                "a kernel gave up a bounded internal wait (error word %d); the step it belonged to was "
+                "skipped; the word stays set until zero_workspace_init",
+                h.error);
   return ZERO_OK;
 }
 
@@ -991,6 +996,10 @@ namespace {
 constexpr int kNoAllocTile = zb::kThreads * 8;  // elements per CTA: one 16-byte vector per thread
 constexpr size_t kNoAllocHeader = 256;          // arrival counter, padded to the array alignment
 constexpr size_t kNoAllocBytes = kNoAllocHeader + sizeof(zb::Partial) * ZERO_NOALLOC_MAX_CTAS;
+// The window limit the header publishes is exactly the CTA count that has scratch slots: a
+// window it accepts never launches more CTAs than there are partial slots.
+static_assert(ZERO_NOALLOC_MAX_WINDOW == (int64_t)ZERO_NOALLOC_MAX_CTAS * kNoAllocTile,
+              "ZERO_NOALLOC_MAX_WINDOW must equal ZERO_NOALLOC_MAX_CTAS x elements per CTA");
 
 // Shared by every call on a device; held by every GPU that loads the library until exit.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
@@ -1125,7 +1134,7 @@ extern "C" int zero_reduce_scatter_noalloc(const uint16_t* const* grads, int dty
   if ((rc = check_hp(hp))) return rc;
   if (dtype != ZERO_BF16 && dtype != ZERO_FP16) return fail(ZERO_EINVAL, "dtype=%d", dtype);
   if (hi - lo > ZERO_NOALLOC_MAX_WINDOW)
-    return fail(ZERO_EINVAL,
+    return fail(ZERO_ENOMEM,
                 "window of %lld elements exceeds the no-allocation limit of %lld elements "
                 "(%d scratch slots of %d elements); split it into smaller windows",
                 (long long)(hi - lo), (long long)ZERO_NOALLOC_MAX_WINDOW, ZERO_NOALLOC_MAX_CTAS, kNoAllocTile);

@@ -2,13 +2,19 @@
 // and per-rank communication volume of plain data parallelism and ZeRO stages 1-3.
 #include "zero.h"
 
+int zero_internal_fail(int code, const char* msg);  // zero_abi.cu: sets zero_last_error
+
 extern "C" {
 
 // [P1] §二 code: weights and gradients take bytes_per_param each, Adam's fp32 copy + m + v take
 // bytes_per_opt_state; ZeRO-1 shards the optimizer state, ZeRO-2 also the gradients, ZeRO-3
 // the weights too.  Results in GiB (2^30 bytes), as the page's helper reports them.
 int zero_memory_estimate(double N, int Nd, int bytes_per_param, int bytes_per_opt_state, zero_mem_t out[4]) {
-  if (!out || !(N >= 0) || Nd < 1 || bytes_per_param < 0 || bytes_per_opt_state < 0) return ZERO_EINVAL;
+  if (!out) return zero_internal_fail(ZERO_EINVAL, "out is NULL");
+  if (!(N >= 0)) return zero_internal_fail(ZERO_EINVAL, "N must be >= 0");
+  if (Nd < 1) return zero_internal_fail(ZERO_EINVAL, "Nd must be >= 1");
+  if (bytes_per_param < 0 || bytes_per_opt_state < 0)
+    return zero_internal_fail(ZERO_EINVAL, "bytes_per_param and bytes_per_opt_state must be >= 0");
   const double gib = 1073741824.0;
   const double weights = N * bytes_per_param / gib;
   const double grads = N * bytes_per_param / gib;
