@@ -5,14 +5,17 @@ One step = one ``zero_step`` call through the C ABI: the reduce-scatter of Nd gr
 replicas, the fp16/bf16 unscale and overflow check, Adam/AdamW on every rank's fp32 shard,
 and the bf16 all-gather to the Nd weight replicas, all Nd simulated ranks in this GPU's memory.
 
-Default workload: ZeRO-1 on N = 124,439,808 parameters (GPT-2 small), Nd = 8 simulated ranks,
-bf16 gradients ~N(0,1e-3), AdamW (lr 6e-4, wd 0.01).  Inputs are synthetic, generated on the
-device by the seeded generator before the timed region (distinct gradients per step, cycling
-through as many sets as fit a memory budget); every step reads more than the 126 MB L2.
+Default workload: the fused reduce-scatter + AdamW + all-gather step on N = 2^28 parameters
+with Nd = 8 simulated ranks, bf16 gradients ~N(0,1e-3), AdamW (lr 1e-3, wd 0.01).  Inputs are
+synthetic, generated on the device by the seeded generator before the timed region (distinct
+gradients per step, cycling through as many sets as fit a memory budget); every step reads more
+than the 126 MB L2.
 
-Prints one JSON line (rank 0).  Under torchrun each rank runs an independent replica of the
-workload on its own GPU (the simulated ranks are already inside one GPU; there is no data-path
-collective), so per-GPU work is fixed (weak scaling) and the value is the sum over GPUs.
+Prints one JSON line (rank 0).  Under torchrun (N > 1 GPUs) the ranks are real data-parallel
+ranks, one per GPU: rank r owns shard r of the workload's parameters and the fused kernel reads
+the peers' gradients and writes every peer's weights over NVLink (zero_sharded_optimizer_03_b200
+.dist); the total work is fixed (strong scaling).  Workloads the real-rank path does not cover
+(ZeRO-3 layers, offload) run one independent replica per GPU instead (weak scaling).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 """
@@ -73,7 +76,7 @@ WORKLOADS = {
         sigma=1e-3, kind="normal",
         hp=dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01, loss_scale=1.0)),
 }
-DEFAULT = "zero1-gpt2-small"
+DEFAULT = "zero2-2p28-nd8"
 
 
 def bytes_per_param(w, two_pass=False, g16=False, fused_layers=False) -> int:
@@ -92,12 +95,31 @@ def bytes_per_param(w, two_pass=False, g16=False, fused_layers=False) -> int:
     return 2 * Nd + 24 + 2 * Nd
 
 
+# NVLink figures for the real-rank roofline: a peer copy measured on this machine's B200s (per
+# direction per GPU) and NVIDIA's nominal link rate, used when MEASURED_PEAKS.json has none.
+NVLINK_PEER_COPY_GBS = 770.0
+NVLINK_NOMINAL_GBS = 900.0
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def nvlink_peak():
+    """(GB/s per direction per GPU, source) for NVLink: MEASURED_PEAKS.json if it has a figure,
+    else the machine's measured peer copy."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        for key in ("nvlink_gbs", "nvlink_peer_gbs", "p2p_gbs"):
+            if key in d:
+                return float(d[key]), "measured (MEASURED_PEAKS.json %s)" % key
+    return NVLINK_PEER_COPY_GBS, ("peer copy measured on this pool, per direction (nominal %g)"
+                                  % NVLINK_NOMINAL_GBS)
 
 
 def traffic_record(kernel: str, workload: str):
@@ -167,9 +189,23 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU baseline
 
-def cpu_baseline(w, target_s=10.0, steps=None):
-    """Time the CPU oracle (single thread, as it stands) on a bounded sample of the workload:
-    the first n parameters, n sized for about target_s seconds of oracle work."""
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, target_s=10.0, steps=1, threads=1, max_bytes=6e9):
+    """Time the CPU oracle as it stands on a bounded sample of the workload: the first n
+    parameters, split into `threads` contiguous chunks of equal length; each thread runs the
+    unmodified, single-threaded oracle step on its own chunk (elements are independent, and the
+    sample has no overflow, so every chunk updates exactly as the whole vector would).  n is
+    sized for about target_s seconds per step and at most max_bytes of host inputs.  Returns
+    (n, [seconds of each step])."""
+    from concurrent.futures import ThreadPoolExecutor
+
     import numpy as np
 
     import oracle
@@ -177,16 +213,23 @@ def cpu_baseline(w, target_s=10.0, steps=None):
     Nd = w["Nd"]
     odt = oracle.FP16 if w["gdt"] == "fp16" else oracle.BF16
     sdt = synth.FP16 if w["gdt"] == "fp16" else synth.BF16
+    kind = synth.HEAVY if w["kind"] == "heavy" else synth.NORMAL
+    tail = float(np.float32(w["sigma"] * 1e3)) if w["kind"] == "heavy" else 0.0
+    t0 = w.get("t0", 0)
 
-    def make(n):
-        grads = [synth.fill_host(synth.NORMAL, sdt, synth.SEED, synth.grad_stream(1, r), n,
-                                 sigma=w["sigma"]) for r in range(Nd)]
-        S, Np, _ = oracle.partition(n, Nd)
-        p = np.zeros(Np, np.float32)
-        p[:n] = synth.fill_host(synth.NORMAL, synth.F32, synth.SEED, synth.MASTER_STREAM, n,
-                                sigma=0.02)
-        return grads, p, np.zeros(Np, np.float32), np.zeros(Np, np.float32), [
-            np.zeros(n, np.uint16) for _ in range(Nd)]
+    def make(lo, n):  # inputs of elements lo .. lo+n-1 (n a multiple of Nd: no padding)
+        grads = [synth.fill_host(kind, sdt, synth.SEED, synth.grad_stream(1, r), n,
+                                 sigma=w["sigma"], tail_sigma=tail, first=lo) for r in range(Nd)]
+        p = synth.fill_host(synth.NORMAL, synth.F32, synth.SEED, synth.MASTER_STREAM, n,
+                            sigma=0.02, first=lo)
+        if t0:
+            m = synth.fill_host(synth.ABS, synth.F32, synth.SEED, synth.M_STREAM, n, sigma=1e-3,
+                                first=lo)
+            v = synth.fill_host(synth.SQUARE, synth.F32, synth.SEED, synth.V_STREAM, n,
+                                sigma=1e-6, first=lo)
+        else:
+            m, v = np.zeros(n, np.float32), np.zeros(n, np.float32)
+        return [grads, p, m, v, [np.zeros(n, np.uint16) for _ in range(Nd)]]
 
     def one_step(n, g, p, m, v, reps, t):
         if w["stage"] == 3:  # the sample is one layer: gather, reduce-scatter, Adam + cast
@@ -197,21 +240,37 @@ def cpu_baseline(w, target_s=10.0, steps=None):
         return oracle.zero12_step(Nd, n, bucket, odt, g, p, m, v, reps, w["hp"], t)[0]
 
     n0 = 1 << 16
-    g, p, m, v, reps = make(n0)
-    t = time.perf_counter()
-    one_step(n0, g, p, m, v, reps, 0)
-    rate0 = n0 / (time.perf_counter() - t)
-    n = int(min(w["N"], max(1 << 12, rate0 * target_s)))
-    if w["stage"] == 3:
-        n -= n % Nd  # one unpadded layer
-    g, p, m, v, reps = make(n)
-    times = []
-    tcount = 0
-    for _ in range(steps or 1):
-        t0 = time.perf_counter()
-        tcount = one_step(n, g, p, m, v, reps, tcount)
-        times.append(time.perf_counter() - t0)
-    return n, times
+    d0 = make(0, n0)
+    tt = time.perf_counter()
+    one_step(n0, *d0, t0)
+    rate0 = n0 / (time.perf_counter() - tt)
+    host_bytes = 4 * Nd + 12 + (2 if w["stage"] == 3 else 0)
+    n = int(min(w["N"], rate0 * target_s * threads, max_bytes / host_bytes))
+    unit = threads * Nd
+    nc = max(1, n // unit) * Nd  # elements per thread
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        data = list(ex.map(lambda c: make(c * nc, nc), range(threads)))
+        tcount = [t0] * threads
+        times = []
+        for _ in range(steps):
+            tt = time.perf_counter()
+            tcount = list(ex.map(lambda c: one_step(nc, *data[c], tcount[c]), range(threads)))
+            times.append(time.perf_counter() - tt)
+    return nc * threads, times
+
+
+def cpu_baseline_record(w, target_s=10.0):
+    """The cpu_baseline object of the bench line: the oracle on every host core (primary) and
+    on one core, each on its own bounded sample of the workload."""
+    ncores = host_threads()
+    n1, t1 = cpu_baseline(w, target_s=target_s, threads=1)
+    nA, tA = cpu_baseline(w, target_s=target_s / 2, threads=ncores)
+    return {"value": nA / tA[0], "unit": "params/s", "cores": ncores, "kind": "oracle",
+            "sample": "first %d of %d parameters, Nd=%d, one ZeRO step, %d contiguous chunks, "
+                      "one oracle call per core (%.1f s)" % (nA, w["N"], w["Nd"], ncores, tA[0]),
+            "single_core": {"value": n1 / t1[0], "unit": "params/s", "cores": 1,
+                            "sample": "first %d of %d parameters, Nd=%d, one ZeRO step (%.1f s)"
+                                      % (n1, w["N"], w["Nd"], t1[0])}}
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -276,10 +335,7 @@ def run_offload(args, w, world, rank, dist, dev, config):
     ms = ms_total / steps
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, times = cpu_baseline(w)
-        cpu = {"value": n / times[0], "unit": "params/s", "cores": 1, "kind": "oracle",
-               "sample": "first %d of %d parameters, Nd=%d, one ZeRO step (%.1f s)"
-               % (n, N, Nd, times[0])}
+        cpu = cpu_baseline_record(w)
     host_bytes = 30 * N  # grad 4 read, master/m/v 12 read + 12 written, bf16 weights 2 written
     pcie_bytes = 6 * N   # fp32 gradient down (4), bf16 weights up (2)
     if rank == 0:
@@ -345,6 +401,10 @@ def run_dist(args, w, config):
         b.record()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    gpu_id = getattr(torch.cuda.get_device_properties(dev), "uuid", None)
+    sampler = ClockSampler(("GPU-" + str(gpu_id)) if gpu_id else str(local))
+    sampler.start()
+    time.sleep(0.3)
     dist.barrier()
     torch.cuda.synchronize()
     t0.record()
@@ -354,33 +414,66 @@ def run_dist(args, w, config):
     t1.record()
     torch.cuda.synchronize()
     dist.barrier()
+    clocks = sampler.stop()
     ms_total, kern_ms = max_over_ranks(
         [t0.elapsed_time(t1), sum(a.elapsed_time(b) for a, b in kev) / args.steps], dist, dev)
     res = dz.result()
     assert res["overflow"] == 0, res
     ms = ms_total / args.steps
+    # end to end, host to host: this rank's gradient replica up from pinned host memory, the
+    # step, this rank's updated bf16 weight replica back to pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        host_g = torch.empty(N, dtype=dz.grad.dtype, pin_memory=True)
+        host_g.copy_(dz.grad)
+        host_p = torch.empty(N, dtype=torch.bfloat16, pin_memory=True)
+        torch.cuda.synchronize()
+        e_start = torch.cuda.Event(enable_timing=True)
+        e_stop = torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        e_start.record()
+        for _ in range(args.e2e_steps):
+            dz.grad.copy_(host_g, non_blocking=True)
+            dz.step(hp)
+            host_p.copy_(dz.param, non_blocking=True)
+            res_e = dz.result()
+            assert res_e["overflow"] == 0, res_e
+        e_stop.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks([e_start.elapsed_time(e_stop)], dist, dev)[0]
+        e2e = {"value": N / (e_ms / args.e2e_steps / 1e3), "unit": "params/s",
+               "h2d_bytes_per_step": 2 * N * world, "d2h_bytes_per_step": (2 * N + 112) * world,
+               "steps": args.e2e_steps, "result": "every rank's bf16 weight replica + step record"}
     S = dz.S
     hbm_bytes = S * (2 + 24 + 2)                   # own gradient, state, own replica (per rank)
     link_bytes = S * 2 * (world - 1) * 2           # peers' gradients in + weights out
-    t_hbm = hbm_bytes / 6527.8e9
-    t_link = link_bytes / 770e9
+    hbm_peak, hbm_src = peaks()
+    link_peak, link_src = nvlink_peak()
+    t_hbm = hbm_bytes / (hbm_peak * 1e9)
+    t_link = link_bytes / (link_peak * 1e9)
     bound = "nvlink" if t_link > t_hbm else "hbm"
     ideal = max(t_hbm, t_link)
     if rank == 0:
         config.update({"Nd": world, "path": "real ranks: fused kernel over peer memory + NCCL "
                        "step totals", "kernel": "fused_step_kernel (peer loads/stores)",
-                       "parallelism": "dp%d (one rank per GPU)" % world})
+                       "parallelism": "dp%d (one rank per GPU)" % world,
+                       "l2": "inputs larger than L2 (%.2f GB gradient replica per rank)"
+                             % (2 * N / 1e9)})
         line = {"metric": METRIC, "value": N / (ms / 1e3), "unit": "params/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
                 "dtype": "f32", "data": "synthetic", "config": config,
                 "roofline": {"bound": bound, "achieved": (hbm_bytes if bound == "hbm" else
                                                           link_bytes) / (kern_ms / 1e3) / 1e9,
-                             "peak": 6527.8 if bound == "hbm" else 770.0, "unit": "GB/s",
+                             "peak": hbm_peak if bound == "hbm" else link_peak, "unit": "GB/s",
                              "frac": ideal / (kern_ms / 1e3), "traffic": None,
+                             "peak_source": hbm_src if bound == "hbm" else link_src,
+                             "hbm_peak": hbm_peak, "hbm_peak_source": hbm_src,
+                             "nvlink_peak": link_peak, "nvlink_peak_source": link_src,
                              "kernel_ms": kern_ms, "hbm_bytes_per_rank": hbm_bytes,
                              "nvlink_bytes_per_rank": link_bytes},
-                "cpu_baseline": None, "e2e": None, "clocks": None,
+                "cpu_baseline": None, "e2e": e2e, "clocks": clocks,
                 "gpu_launches": 3 * args.steps}
         print(json.dumps(line), flush=True)
     dz.close()
@@ -451,16 +544,21 @@ def main():
               % w["Nd"], "l2": "inputs larger than L2 (%.1f GB of gradients per step)"
               % (2 * w["Nd"] * w["N"] / 1e9)}
 
-    if args.dist and args.impl != "reference":
+    # one rank per GPU: the real data-parallel path for flat ZeRO-1/2 workloads
+    real_ranks = world > 1 and w["stage"] in (1, 2) and not w.get("offload")
+    if (args.dist or real_ranks) and args.impl != "reference":
         return run_dist(args, w, config)
 
     if args.impl == "reference":
         if rank != 0:
             return
         # each step is a bounded sample of the workload, sized so that the whole run of
-        # warmup + steps oracle steps takes about two minutes (at most 3 s per step)
+        # warmup + steps oracle steps takes about two minutes (at most 3 s per step); the
+        # oracle runs on every host core, one contiguous chunk of the sample per core
         per_step = min(3.0, 120.0 / (args.warmup + args.steps))
-        n, times = cpu_baseline(w, target_s=per_step, steps=args.warmup + args.steps)
+        cores = host_threads()
+        n, times = cpu_baseline(w, target_s=per_step, steps=args.warmup + args.steps,
+                                threads=cores)
         timed = times[args.warmup:]
         ms = 1e3 * sum(timed) / len(timed)
         val = n / (ms / 1e3)
@@ -468,8 +566,10 @@ def main():
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,
-                "cpu_baseline": {"value": val, "unit": "params/s", "cores": 1, "kind": "oracle",
-                                 "sample": "first %d of %d parameters, Nd=%d, one step each"
+                "cpu_baseline": {"value": val, "unit": "params/s", "cores": cores,
+                                 "kind": "oracle",
+                                 "sample": "first %d of %d parameters, Nd=%d, one step each, "
+                                           "one contiguous chunk per core"
                                  % (n, w["N"], w["Nd"])},
                 "e2e": {"value": val, "unit": "params/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -612,14 +712,20 @@ def main():
         tr = traffic_record(line_kernel, args.workload)
     traffic = tr["dram_bytes_per_launch"] if tr else None
 
-    # end to end through the public API: pinned host gradients -> device, step, result -> host
+    # end to end through the public API, host to host: every step copies the Nd gradient
+    # replicas from pinned host memory to the device, runs the step, copies the step's product
+    # -- the updated bf16 weights (rank 0's replica; for ZeRO-3 the weight shards, which hold
+    # the whole vector) -- back to pinned host memory, and reads the step's bookkeeping
+    # (zero_read_result: overflow / skip, 112 bytes, synchronizing)
     e2e = None
     if not args.no_e2e:
         host = [torch.empty(glen, dtype=buf.grads[0].dtype, pin_memory=True) for _ in range(Nd)]
         for r in range(Nd):
             host[r].copy_(buf.grads[r])
+        result_dev = buf.param_shard if stage == 3 else buf.params[0]
+        result_host = torch.empty(result_dev.numel(), dtype=result_dev.dtype, pin_memory=True)
         torch.cuda.synchronize()
-        res_bytes = 112  # the workspace header zero_read_result copies back
+        d2h = result_dev.numel() * result_dev.element_size() + 112
         e_start = torch.cuda.Event(enable_timing=True)
         e_stop = torch.cuda.Event(enable_timing=True)
         if dist:
@@ -627,23 +733,25 @@ def main():
         torch.cuda.synchronize()
         e_start.record(s)
         for k in range(args.e2e_steps):
+            # (ZeRO-3: the gradient buffers hold one layer, which every layer of the step reuses)
             for r in range(Nd):
                 buf.grads[r].copy_(host[r], non_blocking=True)
             zero.zero_step(stage, Nd, N, w["bucket"], buf.state, hp, sp)
-            zero.zero_read_result(buf.ws.data_ptr(), sp)
+            result_host.copy_(result_dev, non_blocking=True)
+            res_e = zero.zero_read_result(buf.ws.data_ptr(), sp)
+            assert res_e["overflow"] == 0, res_e
         e_stop.record(s)
         torch.cuda.synchronize()
         e_ms = max_over_ranks([e_start.elapsed_time(e_stop)], dist, dev)[0]
         e2e = {"value": whole_job_rate(N, world, e_ms / args.e2e_steps), "unit": "params/s",
-               "h2d_bytes_per_step": 2 * Nd * glen, "d2h_bytes_per_step": res_bytes,
-               "steps": args.e2e_steps}
+               "h2d_bytes_per_step": 2 * Nd * glen,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "result": "bf16 weights (%s) + 112-byte step record" %
+                         ("weight shards, N elements" if stage == 3 else "rank 0 replica, N elements")}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, times = cpu_baseline(w)
-        cpu = {"value": n / times[0], "unit": "params/s", "cores": 1, "kind": "oracle",
-               "sample": "first %d of %d parameters, Nd=%d, one ZeRO step (%.1f s)"
-               % (n, N, Nd, times[0])}
+        cpu = cpu_baseline_record(w)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,

@@ -43,7 +43,21 @@ def test_workloads_match_their_descriptions():
     assert (w["zero2-wide-fanin-nd64"]["N"], w["zero2-wide-fanin-nd64"]["Nd"]) == (1 << 28, 64)
     z3 = w["zero3-llama7b"]
     assert z3["layer"] == 4 * 4096 * 4096 + 3 * 4096 * 11008 and z3["N"] == 32 * z3["layer"]
-    assert bench.DEFAULT == "zero1-gpt2-small"
+    assert bench.DEFAULT == "zero2-2p28-nd8"
+    assert (w[bench.DEFAULT]["N"], w[bench.DEFAULT]["Nd"], w[bench.DEFAULT]["bucket"]) == (1 << 28, 8, 0)
+
+
+def test_cpu_baseline_record_has_the_all_core_and_single_core_legs():
+    """The CPU baseline reports the oracle on every host core (one contiguous chunk per core) and
+    on one core, each with its core count and sample."""
+    w = dict(bench.WORKLOADS["zero2-1m-nd4"])
+    rec = bench.cpu_baseline_record(w, target_s=0.2)
+    assert rec["kind"] == "oracle" and rec["unit"] == "params/s" and rec["value"] > 0
+    assert rec["cores"] == bench.host_threads() >= 1
+    one = rec["single_core"]
+    assert one["cores"] == 1 and one["value"] > 0 and one["sample"]
+    n, times = bench.cpu_baseline(w, target_s=0.05, steps=2, threads=3)
+    assert n % (3 * w["Nd"]) == 0 and 0 < n <= w["N"] and len(times) == 2
 
 
 def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):

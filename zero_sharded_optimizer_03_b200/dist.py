@@ -59,16 +59,22 @@ class DistZero:
             overflowed)
     """
 
-    def __init__(self, N: int, group=None, grad_dtype: int = ZERO_BF16):
+    def __init__(self, N: int, group=None, grad_dtype: int = ZERO_BF16, device=None,
+                 symm=None):
+        """device: this rank's GPU (default: the current CUDA device).  symm: the module that
+        allocates the peer-mapped buffers (default torch.distributed._symmetric_memory; its
+        `empty` and `rendezvous` are all that is used)."""
         import torch
         import torch.distributed as dist
-        import torch.distributed._symmetric_memory as symm
+        if symm is None:
+            import torch.distributed._symmetric_memory as symm
         self.torch, self.dist, self.group = torch, dist, group
         self.N = N
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         self.lo, self.hi, self.S = rank_window(N, self.world, self.rank)
-        dev = torch.device("cuda", torch.cuda.current_device())
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self.device = torch.device(dev)
         gdt = torch.bfloat16 if grad_dtype == ZERO_BF16 else torch.float16
         n = max(N, 1)
         self.grad = symm.empty(n, dtype=gdt, device=dev)
@@ -99,6 +105,8 @@ class DistZero:
         self.state = st
 
     def stream(self) -> int:
+        if self.device.type != "cuda":
+            return 0
         return self.torch.cuda.current_stream().cuda_stream
 
     def init(self, t: int = 0) -> None:
