@@ -42,6 +42,26 @@ def rank_window(N: int, world: int, rank: int):
     return lo, hi, S
 
 
+def shard_state(S: int, lo: int, device, torch):
+    """This rank's fp32 state: two copies each of master / exp_avg / exp_avg_sq for a shard of S
+    elements that starts at global index lo, zero-filled.  Returns (views, bases): views[name][k]
+    is copy k's S-element tensor; bases[name][k] is the device address of global element 0, so
+    bases + 4*lo addresses the shard's first element (the library indexes the state by global
+    position).  Each copy is allocated 3 floats longer and viewed from offset lo % 4, which
+    makes every base 16-byte aligned whatever lo is, so the kernels' 16-byte vector path runs
+    on every rank's window."""
+    off = lo % 4
+    views, bases = {}, {}
+    for name in ("master", "exp_avg", "exp_avg_sq"):
+        views[name], bases[name] = [], []
+        for _ in range(2):
+            t = torch.zeros(max(S, 1) + 3, dtype=torch.float32, device=device)
+            v = t[off:off + max(S, 1)]
+            views[name].append(v)
+            bases[name].append(v.data_ptr() - 4 * lo)
+    return views, bases
+
+
 def combine_step_totals(flag, sumsq, group=None) -> None:
     """Combine the ranks' pending overflow flags (MAX) and sums of squares (SUM) in place."""
     import torch.distributed as dist
@@ -82,11 +102,9 @@ class DistZero:
         gname = (group or dist.group.WORLD).group_name
         self._hg = symm.rendezvous(self.grad, gname)
         self._hp = symm.rendezvous(self.param, gname)
-        s = max(self.S, 1)
-        f32 = dict(dtype=torch.float32, device=dev)
-        self.master = [torch.zeros(s, **f32) for _ in range(2)]
-        self.exp_avg = [torch.zeros(s, **f32) for _ in range(2)]
-        self.exp_avg_sq = [torch.zeros(s, **f32) for _ in range(2)]
+        views, bases = shard_state(self.S, self.lo, dev, torch)
+        self.master, self.exp_avg, self.exp_avg_sq = (views[k] for k in
+                                                      ("master", "exp_avg", "exp_avg_sq"))
         self.ws = torch.zeros(zero_workspace_bytes(), dtype=torch.uint8, device=dev)
         self.flag = self.ws[PENDING_FLAG_OFFSET:PENDING_FLAG_OFFSET + 4].view(torch.int32)
         self.sumsq = self.ws[PENDING_SUMSQ_OFFSET:PENDING_SUMSQ_OFFSET + 8].view(torch.float64)
@@ -98,9 +116,9 @@ class DistZero:
             st.grads[q] = int(self._hg.buffer_ptrs[q])
             st.params[q] = int(self._hp.buffer_ptrs[q])
         for k in range(2):  # state indexed by global position: base + lo is its first element
-            st.master[k] = self.master[k].data_ptr() - 4 * self.lo
-            st.exp_avg[k] = self.exp_avg[k].data_ptr() - 4 * self.lo
-            st.exp_avg_sq[k] = self.exp_avg_sq[k].data_ptr() - 4 * self.lo
+            st.master[k] = bases["master"][k]
+            st.exp_avg[k] = bases["exp_avg"][k]
+            st.exp_avg_sq[k] = bases["exp_avg_sq"][k]
         st.workspace = self.ws.data_ptr()
         self.state = st
 
