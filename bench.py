@@ -95,6 +95,8 @@ def bytes_per_param(w, two_pass=False, g16=False, fused_layers=False) -> int:
     return 2 * Nd + 24 + 2 * Nd
 
 
+L2_BYTES = 126e6  # B200 L2 capacity
+
 # NVLink figures for the real-rank roofline: a peer copy measured on this machine's B200s (per
 # direction per GPU) and NVIDIA's nominal link rate, used when MEASURED_PEAKS.json has none.
 NVLINK_PEER_COPY_GBS = 770.0
@@ -610,7 +612,8 @@ def main():
     tma_path = (not args.two_pass and w["stage"] != 3 and not args.no_tma and
                 (args.tma or (w["Nd"] >= 16 and (w["bucket"] or w["N"]) >= (1 << 24))))
     if w["stage"] == 3 and args.fused_layers:
-        line_kernel = "zero3 step: gather_layer + fused_step kernels (per layer)"
+        line_kernel = ("zero3 step: gather_layer_tma + fused_step kernels (per layer)" if args.tma
+                       else "zero3 step: fused_step kernel with the layer gather (per layer)")
     elif w["stage"] == 3:
         line_kernel = "zero3 step: gather_layer + reduce_scatter + adam kernels"
     elif args.two_pass:
@@ -620,44 +623,67 @@ def main():
     config["kernel"] = line_kernel
     if args.bf16_grad_shard:
         flags |= zero.ZERO_BF16_GRAD_SHARD
-    if stage == 3:
-        assert w["layer"] % Nd == 0 and N % w["layer"] == 0, "unpadded layers expected"
-        buf = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, layer_len=w["layer"],
-                               flags=(zero.ZERO_BF16_GRAD_SHARD if args.bf16_grad_shard else 0)
-                               | (zero.ZERO_FORCE_TMA if args.tma else 0)
-                               | (zero.ZERO_FUSED_LAYERS if args.fused_layers else 0))
-    else:
-        buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt, flags=flags)
-    glen = buf.grads[0].numel()  # N (stages 1/2) or one layer (stage 3, reused per layer)
-    synth.fill_device(buf.master[0].data_ptr(), synth.NORMAL, synth.F32, synth.SEED,
-                      synth.MASTER_STREAM, N, 0.02, cuda_stream=sp)
-    if w.get("t0"):
-        synth.fill_device(buf.exp_avg[0].data_ptr(), synth.ABS, synth.F32, synth.SEED,
-                          synth.M_STREAM, N, 1e-3, cuda_stream=sp)
-        synth.fill_device(buf.exp_avg_sq[0].data_ptr(), synth.SQUARE, synth.F32, synth.SEED,
-                          synth.V_STREAM, N, 1e-6, cuda_stream=sp)
-    buf.init_workspace(w.get("t0", 0))
-    buf.sync_params_from_master()
+    def make_buffers():
+        if stage == 3:
+            assert w["layer"] % Nd == 0 and N % w["layer"] == 0, "unpadded layers expected"
+            b = zero.ZeroBuffers(3, Nd, N, grad_dtype=gdt, layer_len=w["layer"],
+                                 flags=(zero.ZERO_BF16_GRAD_SHARD if args.bf16_grad_shard else 0)
+                                 | (zero.ZERO_FORCE_TMA if args.tma else 0)
+                                 | (zero.ZERO_FUSED_LAYERS if args.fused_layers else 0))
+        else:
+            b = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt, flags=flags)
+        synth.fill_device(b.master[0].data_ptr(), synth.NORMAL, synth.F32, synth.SEED,
+                          synth.MASTER_STREAM, N, 0.02, cuda_stream=sp)
+        if w.get("t0"):
+            synth.fill_device(b.exp_avg[0].data_ptr(), synth.ABS, synth.F32, synth.SEED,
+                              synth.M_STREAM, N, 1e-3, cuda_stream=sp)
+            synth.fill_device(b.exp_avg_sq[0].data_ptr(), synth.SQUARE, synth.F32, synth.SEED,
+                              synth.V_STREAM, N, 1e-6, cuda_stream=sp)
+        b.init_workspace(w.get("t0", 0))
+        b.sync_params_from_master()
+        return b
 
-    # distinct gradient sets (set 0 lives in buf.grads)
+    # A step smaller than a few L2 capacities would find its state and weights still in L2
+    # from its previous run; such workloads cycle through independent optimizer instances (own
+    # state, weights, workspace and gradients) so that every step's data comes from HBM.
+    bpp = bytes_per_param(w, args.two_pass, args.bf16_grad_shard, args.fused_layers)
+    ninst = 1
+    if stage != 3 and bpp * N < 3 * L2_BYTES:
+        ninst = int(min(64, -(-3 * L2_BYTES // (bpp * N))))
+    insts = [make_buffers() for _ in range(ninst)]
+    buf = insts[0]
+    glen = buf.grads[0].numel()  # N (stages 1/2) or one layer (stage 3, reused per layer)
+
+    # distinct gradient sets (set 0 lives in buf.grads; with several instances, instance k's
+    # own buf.grads is set k)
     set_bytes = 2 * Nd * glen
-    nsets = int(max(1, min(args.warmup + args.steps, args.grad_sets_gb * 1e9 // set_bytes)))
-    if stage == 3:
-        nsets = 1
-    gsets = [buf.grads] + [[torch.empty(glen, dtype=buf.grads[0].dtype, device=dev)
-                            for _ in range(Nd)] for _ in range(nsets - 1)]
+    if ninst > 1:
+        nsets = ninst
+        gsets = [b.grads for b in insts]
+    else:
+        nsets = int(max(1, min(args.warmup + args.steps, args.grad_sets_gb * 1e9 // set_bytes)))
+        if stage == 3:
+            nsets = 1
+        gsets = [buf.grads] + [[torch.empty(glen, dtype=buf.grads[0].dtype, device=dev)
+                                for _ in range(Nd)] for _ in range(nsets - 1)]
     states = []
     for k, gs in enumerate(gsets):
         for r in range(Nd):
             synth.fill_device(gs[r].data_ptr(), kind, sdt, synth.SEED,
                               synth.grad_stream(k + 1, r), glen, w["sigma"], tail, cuda_stream=sp)
-        st = zero.zero_state_t.from_buffer_copy(buf.state)
+        st = zero.zero_state_t.from_buffer_copy(insts[k].state if ninst > 1 else buf.state)
         for r in range(Nd):
             st.grads[r] = gs[r].data_ptr()
         states.append(st)
+    if ninst > 1:
+        config["l2"] = ("inputs larger than L2: %d independent optimizer instances cycled, "
+                        "%.0f MB of step data between two runs of one instance"
+                        % (ninst, ninst * bpp * N / 1e6))
     nb = 1 if w["bucket"] == 0 else -(-N // w["bucket"])
     if stage == 3 and args.fused_layers:
-        launches_per_step = 2 * nb + 1  # per layer: gather, fused pass; the overflow-repair check
+        # per layer: the fused gather + update kernel (+ a TMA gather kernel with --tma); the
+        # overflow-repair check
+        launches_per_step = (2 if args.tma else 1) * nb + 1
     elif stage == 3:
         launches_per_step = 3 * nb  # per layer: gather, reduce-scatter, Adam
     elif args.two_pass:
@@ -698,13 +724,13 @@ def main():
     clocks = sampler.stop()
     ms_total = t_start.elapsed_time(t_stop)
     kern_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
-    res = buf.result()
-    assert res["overflow"] == 0 and res["skipped"] == 0, res
+    for b in insts:
+        res = b.result()
+        assert res["overflow"] == 0 and res["skipped"] == 0, res
 
     ms_total, kern_ms = max_over_ranks([ms_total, kern_ms], dist, dev)
     ms_step = ms_total / args.steps
     value = whole_job_rate(N, world, ms_step)
-    bpp = bytes_per_param(w, args.two_pass, args.bf16_grad_shard, args.fused_layers)
     achieved = bpp * N / (kern_ms / 1e3) / 1e9
     peak, peak_src = peaks()
     tr = None
@@ -767,7 +793,7 @@ def main():
                 "hbm_gbs_per_step": bpp * N / (ms_step / 1e3) / 1e9,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
                 "gpu_launches": launches_per_step * args.steps,
-                "grad_sets": nsets}
+                "grad_sets": nsets, "instances": ninst}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()

@@ -37,20 +37,30 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Resident CTAs per SM for each kernel, cached per device (occupancy does not change).
 constexpr int kMaxDevices = 64;
 enum KernelId {
-  kFusedBf16, kFusedFp16, kFusedBf16C1, kFusedFp16C1, kFusedBf16C2, kFusedFp16C2, kFusedBf16C4, kFusedFp16C4, kRsBf16, kRsFp16, kRsBf16Out16, kRsFp16Out16, kAdam, kAdamG16, kCast, kGather,
-  kNumKernels
+  kRsBf16, kRsFp16, kRsBf16Out16, kRsFp16Out16, kAdam, kAdamG16, kCast, kGather,
+  kFusedBase,  // 16 fused-kernel variants: (gather, rank batch 1/2/4/8, gradient dtype)
+  kNumKernels = kFusedBase + 16
 };
 
+// Occupancy id of fused_step_kernel<DT, CH, G>.
+constexpr int ch_index(int CH) { return CH == 1 ? 0 : CH == 2 ? 1 : CH == 4 ? 2 : 3; }
+constexpr int fused_kid(int DT, int CH, bool G) { return kFusedBase + (G ? 8 : 0) + 2 * ch_index(CH) + DT; }
+
+template <int DT, int CH, bool G>
+const void* fused_ptr() {
+  return reinterpret_cast<const void*>(&zb::fused_step_kernel<DT, CH, G>);
+}
+
 const void* kernel_ptr(int id) {
+  if (id >= kFusedBase) {
+    static const void* const table[16] = {
+        fused_ptr<0, 1, false>(), fused_ptr<1, 1, false>(), fused_ptr<0, 2, false>(), fused_ptr<1, 2, false>(),
+        fused_ptr<0, 4, false>(), fused_ptr<1, 4, false>(), fused_ptr<0, 8, false>(), fused_ptr<1, 8, false>(),
+        fused_ptr<0, 1, true>(),  fused_ptr<1, 1, true>(),  fused_ptr<0, 2, true>(),  fused_ptr<1, 2, true>(),
+        fused_ptr<0, 4, true>(),  fused_ptr<1, 4, true>(),  fused_ptr<0, 8, true>(),  fused_ptr<1, 8, true>()};
+    return table[id - kFusedBase];
+  }
   switch (id) {
-    case kFusedBf16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 8>);
-    case kFusedFp16: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 8>);
-    case kFusedBf16C1: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 1>);
-    case kFusedFp16C1: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 1>);
-    case kFusedBf16C2: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 2>);
-    case kFusedFp16C2: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 2>);
-    case kFusedBf16C4: return reinterpret_cast<const void*>(&zb::fused_step_kernel<0, 4>);
-    case kFusedFp16C4: return reinterpret_cast<const void*>(&zb::fused_step_kernel<1, 4>);
     case kRsBf16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0, false>);
     case kRsFp16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<1, false>);
     case kRsBf16Out16: return reinterpret_cast<const void*>(&zb::reduce_scatter_kernel<0, true>);
@@ -242,16 +252,16 @@ void prof_mark(bool start, cudaStream_t s) {
 
 // ------------------------------------------------------------------ launchers
 
-template <int DT, int CH>
-int launch_fused_ch(int kid, zb::FusedArgs a, bool dependent, cudaStream_t s) {
+template <int DT, int CH, bool G>
+int launch_fused_ch(zb::FusedArgs a, bool dependent, cudaStream_t s) {
   int grid = 0;
   const int64_t work = (a.hi - a.lo + 7) / 8;
-  int rc = grid_for(kid, work, &grid);
+  int rc = grid_for(fused_kid(DT, CH, G), work, &grid);
   if (rc) return rc;
   // chunks only for long windows (>= 64 vectors per thread of the wave: on the 25M-element
   // buckets of a 1.3e9-parameter fp16 job at Nd = 16, 16 per thread, they measured 1% slower)
   // and launches whose last CTA resets the counter (mode != 0)
-  a.chunked = a.mode != 0 && work >= 64 * (int64_t)grid * zb::kThreads && use_chunks(a.Nd, a.nrep);
+  a.chunked = a.mode != 0 && work >= 64 * (int64_t)grid * zb::kThreads && use_chunks(a.Nd, G ? a.Nd : a.nrep);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(zb::kThreads);
@@ -266,7 +276,7 @@ int launch_fused_ch(int kid, zb::FusedArgs a, bool dependent, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, zb::fused_step_kernel<DT, CH>, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, zb::fused_step_kernel<DT, CH, G>, a);
   if (e != cudaSuccess) return cuda_fail(e, "fused_step_kernel launch");
   return check_launch("fused_step_kernel launch");
 }
@@ -276,16 +286,18 @@ int launch_fused_ch(int kid, zb::FusedArgs a, bool dependent, cudaStream_t s) {
 // +1.4% to +3.7% with chunks, +3.5% for a single output), else 8.
 // dependent: a later bucket of the same step, launched right after the previous bucket's fused
 // kernel on the same stream (programmatic dependent launch).
-int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s, bool dependent = false) {
+template <bool G>
+int launch_fused_g(int dtype, const zb::FusedArgs& a, cudaStream_t s, bool d) {
   const bool f16 = dtype == ZERO_FP16;
-  const bool d = dependent;
-  if (a.Nd <= 1)
-    return f16 ? launch_fused_ch<1, 1>(kFusedFp16C1, a, d, s) : launch_fused_ch<0, 1>(kFusedBf16C1, a, d, s);
-  if (a.Nd <= 2)
-    return f16 ? launch_fused_ch<1, 2>(kFusedFp16C2, a, d, s) : launch_fused_ch<0, 2>(kFusedBf16C2, a, d, s);
-  if (a.Nd <= 8)
-    return f16 ? launch_fused_ch<1, 4>(kFusedFp16C4, a, d, s) : launch_fused_ch<0, 4>(kFusedBf16C4, a, d, s);
-  return f16 ? launch_fused_ch<1, 8>(kFusedFp16, a, d, s) : launch_fused_ch<0, 8>(kFusedBf16, a, d, s);
+  if (a.Nd <= 1) return f16 ? launch_fused_ch<1, 1, G>(a, d, s) : launch_fused_ch<0, 1, G>(a, d, s);
+  if (a.Nd <= 2) return f16 ? launch_fused_ch<1, 2, G>(a, d, s) : launch_fused_ch<0, 2, G>(a, d, s);
+  if (a.Nd <= 8) return f16 ? launch_fused_ch<1, 4, G>(a, d, s) : launch_fused_ch<0, 4, G>(a, d, s);
+  return f16 ? launch_fused_ch<1, 8, G>(a, d, s) : launch_fused_ch<0, 8, G>(a, d, s);
+}
+
+// a.gsrc != NULL selects the variant that also gathers a ZeRO-3 layer (see fused_step_kernel).
+int launch_fused(int dtype, const zb::FusedArgs& a, cudaStream_t s, bool dependent = false) {
+  return a.gsrc ? launch_fused_g<true>(dtype, a, s, dependent) : launch_fused_g<false>(dtype, a, s, dependent);
 }
 
 // TMA-pipelined fused step over [a.lo, a.hi): whole tiles through the bulk-copy pipeline, the
@@ -461,9 +473,11 @@ void adam_host(float* p, float* m, float* v, const float* g, uint16_t* out16, in
 float clip_factor(double max_norm, double sumsq);
 }  // namespace zh
 
-// ZeRO-3 step with one fused pass per layer (flag ZERO_FUSED_LAYERS): the forward gather of
-// layer l, then the layer's reduce-scatter, unscale, flag / sum of squares, AdamW and bf16 cast
-// in one kernel (the K1 kernel with a single bf16 output: the layer's concatenated shards).  The
+// ZeRO-3 step with one fused pass per layer (flag ZERO_FUSED_LAYERS): the gather of layer l and
+// the layer's reduce-scatter, unscale, flag / sum of squares, AdamW and bf16 cast in one kernel
+// (the K1 kernel with a single bf16 output, the layer's concatenated shards, whose G variant
+// copies each old shard word to the Nd gathered-layer buffers before replacing it; with
+// ZERO_FORCE_TMA the gather is a TMA fan-out kernel of its own before the pass).  The
 // global overflow decision is known only after the last layer, so every layer's update goes into
 // the other state copy (read `live`, write 1 - live) and the bf16 shards are written
 // speculatively; the last layer's launch ends the step and makes the new copy live unless the
@@ -500,15 +514,23 @@ static int zero3_fused_layers(int Nd, int64_t N, int64_t bucket, const zero_stat
       shards[r] = st->param_shard + off + r * Sl;
       outs[r] = st->params[r] + l * st->param_layer_stride;
     }
-    rc = (st->flags & ZERO_FORCE_TMA) ? do_gather_tma(shards, Nd, Ll, outs, Nd, ws, s)
-                                      : do_gather(shards, Nd, Ll, outs, Nd, s);
-    if (rc) return rc;
+    // The gather rides in the fused pass (one kernel per layer, see fused_step_kernel's G
+    // variant) unless ZERO_FORCE_TMA asks for the TMA fan-out as a kernel of its own.
+    const bool tma_gather = (st->flags & ZERO_FORCE_TMA) != 0;
+    if (tma_gather && (rc = do_gather_tma(shards, Nd, Ll, outs, Nd, ws, s))) return rc;
     zb::FusedArgs a;
     std::memset(&a, 0, sizeof a);
     bool fal = true;
     for (int r = 0; r < Nd; ++r) {
       a.grads[r] = st->grads[r] + l * st->grad_layer_stride;
       fal = fal && aligned16(a.grads[r]);
+    }
+    if (!tma_gather) {
+      a.gsrc = st->param_shard + off;
+      for (int r = 0; r < Nd; ++r) {
+        a.gout[r] = outs[r];
+        fal = fal && aligned16(outs[r]);
+      }
     }
     a.reps[0] = st->param_shard + off;
     a.nrep = 1;

@@ -368,7 +368,16 @@ struct FusedArgs {
   int nrep;     // bf16 outputs per element: the Nd replicas (ZeRO-1/2), or 1 (a ZeRO-3 layer's shard)
   int chunked;  // 1: CTAs take chunks of kChunkVecs vectors from hdr->chunk (needs mode != 0)
   int trigger_late;  // 1: a dependent launch may start only once this CTA's main loop is done
+  // ZeRO-3 layer with its gather (kernel variant G): gsrc is the layer's bf16 weights before the
+  // update (the concatenated shards, the same memory as reps[0]); each element's old word is
+  // copied to the Nd gathered-layer buffers gout[r] before the new weight overwrites it
+  const uint16_t* gsrc;
+  uint16_t* gout[kMaxNd];
 };
+
+// Compiler-only ordering point: memory accesses written before it are emitted before those
+// written after it (used where a thread reads a word and later overwrites the same word).
+__device__ __forceinline__ void compiler_fence() { asm volatile("" ::: "memory"); }
 
 // Programmatic dependent launch: a grid launched with programmatic stream serialization may
 // start while the previous grid in the stream finishes.  launch_dependents lets the next grid
@@ -398,7 +407,12 @@ constexpr int64_t kChunkVecs = (int64_t)kChunkIters * kThreads;
 // only): the next bucket's CTAs start streaming while this one's last CTAs finish.  The header
 // fields read at the start (t, live, loss scale) change only when a step ends, and a dependent
 // grid waits for its predecessor before it touches the partials and the counters.
-template <int DT, int CH>
+//
+// G (ZeRO-3 layer with its gather): every element j of the layer is also the layer's gathered
+// weight j (the gather concatenates the Nd shards, which lie back to back), so one pass reads
+// the old bf16 word, fans it out to the Nd gathered buffers, and then writes the updated
+// weight over it: 2 + 2Nd bytes of gather traffic ride along with the update's 26 + 2Nd.
+template <int DT, int CH, bool G = false>
 __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   __shared__ Bias s_bias;
   __shared__ int s_live;
@@ -429,10 +443,16 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
   auto vector_step = [&](int64_t j) {
     const int64_t i = sp8.vlo + (j << 3);
     float P[8], M[8], V[8], s[8];
+    uint4 w_old;
+    if (G) w_old = ld_stream(a.gsrc + i);
     unpack(ld_stream(sp + i), ld_stream(sp + i + 4), P);
     unpack(ld_stream(sm + i), ld_stream(sm + i + 4), M);
     unpack(ld_stream(sv + i), ld_stream(sv + i + 4), V);
     fan_in8<DT, CH>(a.grads, a.Nd, i, s);
+    if (G) {  // the gather: the old weights to every rank's layer buffer, before they are replaced
+      for (int r = 0; r < a.Nd; ++r) st_stream(a.gout[r] + i, w_old);
+      compiler_fence();
+    }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const float g = __fmul_rn(s[k], inv);
@@ -475,6 +495,11 @@ __global__ void __launch_bounds__(kThreads, CH <= 4 ? 3 : 2) fused_step_kernel(c
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < sp8.nrest; e += stride) {
     const int64_t i = sp8.scalar_index(a.lo, e);
+    if (G) {
+      const uint16_t w_old = a.gsrc[i];
+      for (int r = 0; r < a.Nd; ++r) a.gout[r][i] = w_old;
+      compiler_fence();
+    }
     const float g = __fmul_rn(fan_in1<DT>(a.grads, a.Nd, i), inv);
     bad |= nonfinite(g);
     sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
