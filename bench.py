@@ -506,9 +506,16 @@ def main():
     ap.add_argument("--bf16-grad-shard", action="store_true",
                     help="two-pass / stage 3: keep the reduced gradient as bf16")
     ap.add_argument("--two-pass", action="store_true",
-                    help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather")
+                    help="stages 1/2: reduce-scatter into an fp32 shard, then Adam + all-gather; "
+                         "stage 3: the two-phase step (gathers and reduce-scatters, then Adam)")
     ap.add_argument("--fused-layers", action="store_true",
-                    help="stage 3: one speculative fused pass per layer (two fp32 state copies)")
+                    help="stage 3: one speculative fused pass per layer carrying the layer's "
+                         "gather (two fp32 state copies); the default for stage 3 unless "
+                         "--two-pass or --bf16-grad-shard")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay the timed steps from CUDA graphs (default for launch-bound steps)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every timed step from the host, even a launch-bound one")
     ap.add_argument("--bucket-override", type=int, default=-1,
                     help="stages 1/2: run with a different bucket size (0 = one bucket)")
     ap.add_argument("--nd-override", type=int, default=0,
@@ -520,6 +527,12 @@ def main():
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     w = dict(WORKLOADS[args.workload])
+    if w["stage"] == 3 and not args.two_pass and not args.bf16_grad_shard:
+        # the faster ZeRO-3 step (60 B/param against 68) whenever its second fp32 state copy fits
+        # (the Llama-7B-shaped job: 155 GB of state + 6.5 GB of layer buffers of 180 GB)
+        args.fused_layers = True
+    if w["stage"] == 3 and args.two_pass:
+        args.two_pass, args.fused_layers = False, False  # stage 3's two-phase step
     if args.n_override:
         w["N"] = args.n_override
         w["desc"] += " [N overridden to %d]" % args.n_override
@@ -700,6 +713,42 @@ def main():
         step(k)
     torch.cuda.synchronize()
 
+    # Launch-bound steps (the workloads that cycle optimizer instances: tens of microseconds per
+    # step) are replayed from CUDA graphs of captured zero_step calls, as a training loop of
+    # such a model would run them: the host cost of a Python call and two kernel launches per
+    # step is then paid once at capture.  One graph holds one step of every instance in order;
+    # single-step graphs make up a remainder, so exactly args.steps steps are timed.
+    use_graph = (ninst > 1 and not args.no_graph) or args.graph
+    graphs_all, graphs_one = None, []
+    if use_graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(s)
+        for k in range(nsets):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                zero.zero_step(stage, Nd, N, w["bucket"], states[k], hp, side.cuda_stream)
+            graphs_one.append(g)
+        graphs_all = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graphs_all, stream=side):
+            for k in range(nsets):
+                zero.zero_step(stage, Nd, N, w["bucket"], states[k], hp, side.cuda_stream)
+        s.wait_stream(side)
+        for _ in range(2):  # warm replays (capture runs nothing)
+            graphs_all.replay()
+        torch.cuda.synchronize()
+        config["launch"] = ("CUDA graphs of captured zero_step calls (%d steps per graph), "
+                            "replayed" % nsets)
+
+    def timed_steps():
+        if not use_graph:
+            for k in range(args.steps):
+                step(args.warmup + k)
+            return
+        for _ in range(args.steps // nsets):
+            graphs_all.replay()
+        for k in range(args.steps % nsets):
+            graphs_one[k].replay()
+
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     for a, b in kev:  # create the underlying CUDA events before handing them to the library
@@ -715,15 +764,21 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     t_start.record(s)
-    for k in range(args.steps):
-        step(args.warmup + k, kev[k])
+    timed_steps()
     t_stop.record(s)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
+    # the same number of steps again, each bracketed by CUDA events around its data kernels
+    # (the roofline's kernel time); kept out of the loop above, whose time per step is the
+    # headline, because an event record between two steps costs time on a microsecond step
+    for k in range(args.steps):
+        step(args.warmup + args.steps + k, kev[k])
+    torch.cuda.synchronize()
     clocks = sampler.stop()
     ms_total = t_start.elapsed_time(t_stop)
     kern_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
+    del graphs_all, graphs_one
     for b in insts:
         res = b.result()
         assert res["overflow"] == 0 and res["skipped"] == 0, res
