@@ -9,8 +9,10 @@ is decided by OR-ing the chunks' overflow flags from the oracle's own reduce-sca
 inputs of each chunk are regenerated on the host by the seeded counter-based generator.
 
 Workloads: two Llama-7B-shaped ZeRO-3 layers (2 x 202,375,168 elements, Nd = 8) through
-zero_step(stage=3), two-phase and fused-layers, with an overflowing step; and the wide fan-in
-step (2^28 elements, Nd = 64, heavy-tailed bf16 gradients, AdamW step 1000 with prefilled m, v).
+zero_step(stage=3), two-phase and fused-layers, with an overflowing step; the wide fan-in step
+(2^28 elements, Nd = 64, heavy-tailed bf16 gradients, AdamW step 1000 with prefilled m, v); ten
+ZeRO-1 steps of GPT-2 small (124,439,808, Nd = 8); two steps at 2^28, Nd = 8 (the bench's
+default workload); five bucketed fp16 steps of 1.3e9 elements at Nd = 16 with a skipped one.
 """
 from __future__ import annotations
 
@@ -24,7 +26,8 @@ import torch
 import oracle
 import synth
 import zero_sharded_optimizer_03_b200 as zero
-from _gpu import HP_ADAMW_WIDE, HP_ADAMW_ZERO3, LLAMA7B_LAYER, SEED, fill, free, u16
+from _gpu import (HP_ADAMW_FP16_LS1024, HP_ADAMW_GPT2, HP_ADAMW_WIDE, HP_ADAMW_ZERO3, LLAMA7B_LAYER,
+                  SEED, fill, free, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -204,3 +207,97 @@ def test_wide_fan_in_2p28_nd64_every_element():
     assert abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
     del buf
     free()
+
+
+# ----------------------------------------------------------------------------- ZeRO-1/2, several steps
+
+def _zero12_every_element(stage, Nd, N, steps, hp, gdt, sigma, bucket=0, inject=None):
+    """Run `steps` zero_step calls of stage 1/2 (fused path; bucketed if bucket) on the device,
+    then compare the final fp32 state and rank 0's bf16 replica element by element with the
+    oracle run over every chunk for the same steps (the other replicas must equal rank 0's).
+    inject = (step, (rank, index)): +inf planted there; that step must be skipped."""
+    sdt = synth.BF16 if gdt == zero.ZERO_BF16 else synth.FP16
+    odt = oracle.BF16 if gdt == zero.ZERO_BF16 else oracle.FP16
+    inf_bits = 0x7F80 if sdt == synth.BF16 else 0x7C00
+    chp = zero.hparams(**hp)
+    buf = zero.ZeroBuffers(stage, Nd, N, grad_dtype=gdt)
+    assert buf.Np == N  # the workloads here are multiples of Nd: no padding
+    fill(buf.master[0], synth.NORMAL, synth.F32, synth.MASTER_STREAM, n=N, sigma=0.02)
+    buf.init_workspace(0)
+    buf.sync_params_from_master()
+    for k in range(1, steps + 1):
+        for r in range(Nd):
+            fill(buf.grads[r], synth.NORMAL, sdt, synth.grad_stream(k, r), sigma=sigma)
+        if inject and k == inject[0]:
+            buf.grads[inject[1][0]].view(torch.int16)[inject[1][1]] = inf_bits
+        buf.step(chp, bucket=bucket)
+    res = buf.result()
+    skipped = {inject[0]} if inject else set()
+    assert (res["step"], res["skipped"]) == (steps - len(skipped), len(skipped)), res
+    live = buf.live()
+    for r in range(1, Nd):
+        assert torch.equal(buf.params[r].view(torch.int16), buf.params[0].view(torch.int16))
+    got_p = buf.master[live].cpu().numpy()
+    got_m = buf.exp_avg[live].cpu().numpy()
+    got_v = buf.exp_avg_sq[live].cpu().numpy()
+    got_w = u16(buf.params[0])
+    del buf
+    free()
+    chunks = [(lo, min(CHUNK, N - lo)) for lo in range(0, N, CHUNK)]
+    assert all(n % Nd == 0 for _, n in chunks)  # every chunk is its own unpadded partition
+
+    def grads(k, lo, n):
+        g = _grads_chunk(Nd, sdt, k, lo, n, sigma)
+        if inject and k == inject[0]:
+            rank, idx = inject[1]
+            if lo <= idx < lo + n:
+                g[rank][idx - lo] = inf_bits
+        return g
+
+    for k in sorted(skipped):  # the oracle's reduce-scatter decides the skip
+        assert any(_pmap(lambda c: oracle.reduce_scatter(Nd, c[1], odt, grads(k, *c), hp)[1],
+                         chunks)), "the oracle does not skip step %d" % k
+
+    def check(c):
+        lo, n = c
+        p = synth.fill_host(synth.NORMAL, synth.F32, SEED, synth.MASTER_STREAM, n, sigma=0.02,
+                            first=lo)
+        m = np.zeros(n, np.float32)
+        v = np.zeros(n, np.float32)
+        reps = [np.zeros(n, np.uint16) for _ in range(Nd)]
+        t, ss = 0, 0.0
+        for k in range(1, steps + 1):
+            if k in skipped:  # a skipped step changes nothing
+                continue
+            t, ovf, ss = oracle.zero12_step(Nd, n, 0, odt, grads(k, lo, n), p, m, v, reps, hp, t)
+            assert ovf == 0
+        return (f32_err(got_p[lo:lo + n], p), f32_err(got_m[lo:lo + n], m),
+                f32_err(got_v[lo:lo + n], v), bf16_ulps(got_w[lo:lo + n], reps[0]), ss)
+    out = _pmap(check, chunks)
+    worst = np.array([o[:4] for o in out], dtype=np.float64).max(axis=0)
+    assert worst[0] <= 1e-6 and worst[1] <= 1e-6 and worst[2] <= 1e-6, worst
+    assert worst[3] <= 1, worst
+    ss = sum(o[4] for o in out)  # the last step's sum of squares
+    assert abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
+
+
+def test_zero1_gpt2_small_ten_steps_every_element():
+    """N = 124,439,808 (GPT-2 small), Nd = 8, ZeRO-1, 10 AdamW steps (lr 6e-4, wd 0.01), fresh
+    bf16 gradients ~N(0,1e-3) every step, bf16 weights all-gathered to 8 replicas each step."""
+    _zero12_every_element(1, 8, 124_439_808, 10, dict(HP_ADAMW_GPT2), zero.ZERO_BF16, 1e-3)
+
+
+def test_zero2_2p28_nd8_two_steps_every_element():
+    """The default bench workload: N = 2^28, Nd = 8, bf16 gradients ~N(0,1e-3), AdamW (lr 1e-3,
+    wd 0.01), two steps through the fused kernel."""
+    _zero12_every_element(2, 8, 1 << 28, 2, dict(HP_ADAMW_WIDE), zero.ZERO_BF16, 1e-3)
+
+
+def test_zero2_1p3b_fp16_buckets_overflow_every_element():
+    """N = 1.3e9 in 25M-element buckets (52), Nd = 16, fp16 gradients ~N(0,1e-4)*1024 carrying
+    loss scale 1024; +inf at the seeded (rank, index) on step 3, which must be skipped; 5 AdamW
+    steps (the TMA-pipelined kernel at this fan-in)."""
+    N, Nd = 1_300_000_000, 16
+    site = synth.inject_site(SEED, Nd, N)
+    _zero12_every_element(2, Nd, N, 5, dict(HP_ADAMW_FP16_LS1024), zero.ZERO_FP16, 1e-4 * 1024,
+                          bucket=25_000_000, inject=(3, site))

@@ -413,19 +413,20 @@ constexpr int64_t kChunkVecs = (int64_t)kChunkIters * kThreads;
 // the old bf16 word, fans it out to the Nd gathered buffers, and then writes the updated
 // weight over it: 2 + 2Nd bytes of gather traffic ride along with the update's 26 + 2Nd.
 //
-// Start of a launch.  With EARLY (every batch width but 2), every thread reads the live copy
-// index itself (one broadcast load per warp), because the state loads depend on it; the bias
-// corrections and the unscale factor, which thread 0 evaluates in double, are needed only once
-// the data has arrived, so the barrier that publishes them comes after each thread has issued
-// its first vector's loads.  Without EARLY, thread 0 reads the header and evaluates the
-// scalars before a barrier, and only then do the loads start: at batches of 2 (Nd = 2) that
-// order measured 11% faster on 2^28 elements, at 1 and 4-8 replicas the early one 1-2% faster.
+// Start of a launch.  With EARLY (every instantiation but batches of 2 without the gather),
+// every thread reads the live copy index itself (one broadcast load per warp), because the
+// state loads depend on it; the bias corrections and the unscale factor, which thread 0
+// evaluates in double, are needed only once the data has arrived, so the barrier that publishes
+// them comes after each thread has issued its first vector's loads (1-2% faster at 1 and 4-8
+// replicas than waiting for them).  Without EARLY, thread 0 reads the header and evaluates the
+// scalars before a barrier, the loads start after it, and the loop body keeps its vector in
+// registers of its own: at Nd = 2 that form measured faster than the restructured one.
 // Registers are budgeted for 4 resident CTAs per SM at single-replica batches (3 with the
 // gather, which would spill at 64 registers), 3 up to batches of 4 and 2 at 8.
 template <int DT, int CH, bool G = false>
 __global__ void __launch_bounds__(kThreads, (CH <= 1 && !G) ? 4 : CH <= 4 ? 3 : 2) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   constexpr int BT = kThreads;
-  constexpr bool EARLY = CH != 2;
+  constexpr bool EARLY = CH != 2 || G;
   __shared__ Bias s_bias;
   __shared__ float s_inv;
   __shared__ int s_live;
@@ -541,23 +542,50 @@ __global__ void __launch_bounds__(kThreads, (CH <= 1 && !G) ? 4 : CH <= 4 ? 3 : 
   } else {
     const int64_t stride = (int64_t)gridDim.x * BT;
     int64_t j = (int64_t)blockIdx.x * BT + threadIdx.x;
-    Vec R;
     if constexpr (EARLY) {
+      Vec R;
       const bool first = j < sp8.nvec;
       if (first) load(j, R);  // in flight while thread 0 evaluates the step scalars
       __syncthreads();
       b = s_bias;
       inv = s_inv;
       if (first) finish(j, R, b, inv);
-      j += stride;
-    } else {
-      b = s_bias;
-      inv = s_inv;
-    }
 #pragma unroll 1
-    for (; j < sp8.nvec; j += stride) {
-      load(j, R);
-      finish(j, R, b, inv);
+      for (j += stride; j < sp8.nvec; j += stride) {
+        load(j, R);
+        finish(j, R, b, inv);
+      }
+    } else {
+      // one vector per iteration with everything in the loop body's own registers (the same
+      // arithmetic as load + finish, in the loop shape this instantiation measured fastest in)
+      const Bias bb = s_bias;
+      const float ii = s_inv;
+      b = bb;
+      inv = ii;
+#pragma unroll 1
+      for (; j < sp8.nvec; j += stride) {
+        const int64_t i = sp8.vlo + (j << 3);
+        float P[8], M[8], V[8], sg[8];
+        unpack(ld_stream(sp + i), ld_stream(sp + i + 4), P);
+        unpack(ld_stream(sm + i), ld_stream(sm + i + 4), M);
+        unpack(ld_stream(sv + i), ld_stream(sv + i + 4), V);
+        fan_in8<DT, CH>(a.grads, a.Nd, i, sg);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float g = __fmul_rn(sg[k], ii);
+          bad |= nonfinite(g);
+          sq = __dadd_rn(sq, __dmul_rn((double)g, (double)g));
+          adam_elem(g, P[k], M[k], V[k], a.c, bb);
+        }
+        st_stream(dp + i, make_float4(P[0], P[1], P[2], P[3]));
+        st_stream(dp + i + 4, make_float4(P[4], P[5], P[6], P[7]));
+        st_stream(dm + i, make_float4(M[0], M[1], M[2], M[3]));
+        st_stream(dm + i + 4, make_float4(M[4], M[5], M[6], M[7]));
+        st_stream(dv + i, make_float4(V[0], V[1], V[2], V[3]));
+        st_stream(dv + i + 4, make_float4(V[4], V[5], V[6], V[7]));
+        const uint4 w = pack_bf16x8(P);
+        for (int r = 0; r < a.nrep; ++r) st_stream(a.reps[r] + i, w);
+      }
     }
   }
   // before a dependent that only waits for this grid (the overflow-repair check), trigger late:
