@@ -140,6 +140,16 @@ def traffic_record(kernel: str, workload: str):
     return None
 
 
+def optimizer_instances(stage: int, step_bytes: float) -> int:
+    """Independent optimizer instances a workload cycles through so that a step finds none of
+    its data in L2 from its previous run: enough that three L2 capacities of other steps' data
+    pass between two runs of one instance (at most 64); 1 for steps that large already, and for
+    ZeRO-3 (its steps are gigabytes)."""
+    if stage == 3 or step_bytes >= 3 * L2_BYTES:
+        return 1
+    return int(min(64, -(-3 * L2_BYTES // step_bytes)))
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -660,9 +670,7 @@ def main():
     # from its previous run; such workloads cycle through independent optimizer instances (own
     # state, weights, workspace and gradients) so that every step's data comes from HBM.
     bpp = bytes_per_param(w, args.two_pass, args.bf16_grad_shard, args.fused_layers)
-    ninst = 1
-    if stage != 3 and bpp * N < 3 * L2_BYTES:
-        ninst = int(min(64, -(-3 * L2_BYTES // (bpp * N))))
+    ninst = optimizer_instances(stage, bpp * N)
     insts = [make_buffers() for _ in range(ninst)]
     buf = insts[0]
     glen = buf.grads[0].numel()  # N (stages 1/2) or one layer (stage 3, reused per layer)

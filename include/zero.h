@@ -275,9 +275,11 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
  *     weights from param_shard into params[r] (every rank), reduce-scatter its gradient
  *     replicas into grad_shard; after the last layer, if no overflow, Adam in place on copy 0
  *     and param_shard = bf16(master).
- *   stage 3, ZERO_FUSED_LAYERS: for each layer, the gather as above, then one fused pass over
- *     the layer (reduce-scatter of its gradient replicas, unscale, overflow check, Adam from
- *     copy `live` into copy 1-live, and the layer's param_shard = bf16(new master)).  The
+ *   stage 3, ZERO_FUSED_LAYERS: for each layer, one fused pass over the layer that also
+ *     gathers it: each element's old bf16 weight goes to every params[r] (the gather above),
+ *     then the reduce-scatter of its gradient replicas, unscale, overflow check, Adam from copy
+ *     `live` into copy 1-live, and the layer's param_shard = bf16(new master) over the old
+ *     weight (with ZERO_FORCE_TMA the gather is a TMA fan-out kernel before the pass).  The
  *     overflow decision needs every layer, so the updates are speculative: the end of the step
  *     swaps the copies if no element overflowed; otherwise param_shard is rewritten from the
  *     unchanged copy.  Same values as the two-phase stage 3, 28 + 4*Nd bytes of traffic per

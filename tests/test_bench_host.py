@@ -110,3 +110,16 @@ def test_reference_arm_prints_the_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["config"]["workload"] == bench.WORKLOADS[bench.DEFAULT]["desc"]
+
+
+def test_short_workloads_cycle_optimizer_instances():
+    """A step smaller than three L2 capacities cycles independent optimizer instances so that its
+    data comes from HBM: the 1M-element workload (40 B/param) takes 10, the large ones 1."""
+    w = bench.WORKLOADS
+    assert bench.optimizer_instances(2, 40 * w["zero2-1m-nd4"]["N"]) == 10
+    assert bench.optimizer_instances(2, 56 * w["zero2-2p28-nd8"]["N"]) == 1
+    assert bench.optimizer_instances(1, 56 * w["zero1-gpt2-small"]["N"]) == 1
+    assert bench.optimizer_instances(3, 1000) == 1
+    assert bench.optimizer_instances(2, 40 * 8192) == 64
+    n = bench.optimizer_instances(2, 40 * 262_144)
+    assert (n - 1) * 40 * 262_144 < 3 * bench.L2_BYTES <= n * 40 * 262_144
