@@ -757,8 +757,10 @@ def main():
         for k in range(args.steps % nsets):
             graphs_one[k].replay()
 
+    # at least 100 evented steps, so that one slow step does not decide the average
+    kev_steps = max(args.steps, 100)
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+           for _ in range(kev_steps)]
     for a, b in kev:  # create the underlying CUDA events before handing them to the library
         a.record(s)
         b.record(s)
@@ -777,15 +779,17 @@ def main():
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    # the same number of steps again, each bracketed by CUDA events around its data kernels
-    # (the roofline's kernel time); kept out of the loop above, whose time per step is the
-    # headline, because an event record between two steps costs time on a microsecond step
-    for k in range(args.steps):
+    # more steps, each bracketed by CUDA events around its data kernels (the roofline's kernel
+    # time); kept out of the loop above, whose time per step is the headline, because an event
+    # record between two steps costs time on a microsecond step
+    for k in range(kev_steps):
         step(args.warmup + args.steps + k, kev[k])
     torch.cuda.synchronize()
     clocks = sampler.stop()
     ms_total = t_start.elapsed_time(t_stop)
-    kern_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
+    kern_list = [a.elapsed_time(b) for a, b in kev]
+    kern_ms = sum(kern_list) / kev_steps
+    kern_median = statistics.median(kern_list)
     del graphs_all, graphs_one
     for b in insts:
         res = b.result()
@@ -852,6 +856,7 @@ def main():
                              "peak_source": peak_src,
                              "kernel": line_kernel,
                              "bytes_per_param": bpp, "kernel_ms": kern_ms,
+                             "kernel_ms_median": kern_median, "kernel_steps": kev_steps,
                              "frac_of_8TBs": achieved / 8000.0},
                 "hbm_gbs_per_step": bpp * N / (ms_step / 1e3) / 1e9,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,

@@ -267,7 +267,10 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
  *     overflow-repair check after the last, are programmatic dependent launches on `stream`
  *     (each may start while the previous kernel of the step finishes; it waits for that kernel
  *     before using its results), so nothing else should be enqueued between them: one
- *     zero_step call enqueues the whole step.
+ *     zero_step call enqueues the whole step.  The first launch of the register-pipelined pass
+ *     is a programmatic dependent of whatever precedes it on `stream` and waits for it to
+ *     complete before it reads or writes anything, so stream order is kept; after a previous
+ *     step's repair check its launch overlaps that kernel.
  *   stage 1/2, ZERO_TWO_PASS: reduce-scatter into grad_shard, then (if no overflow) Adam in
  *     place on copy 0 fused with the cast and the all-gather.
  *   stage 3: N elements in layers of `bucket` elements (the last may be shorter; bucket = 0

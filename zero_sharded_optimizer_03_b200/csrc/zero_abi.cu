@@ -270,7 +270,7 @@ int launch_fused_ch(zb::FusedArgs a, bool dependent, cudaStream_t s) {
   cudaLaunchAttribute attr[1];
   // a later bucket of the same step may overlap the previous one's tail (fixed split only: the
   // chunk counter is shared between launches)
-  if (dependent && !a.chunked) {
+  if ((dependent && !a.chunked) || a.wait_first) {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
@@ -977,6 +977,10 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     a.hi = (k + 1) * B < N ? (k + 1) * B : N;
     a.mode = (k == 0 ? zb::kAccSet : zb::kAccAdd) | (k == nb - 1 ? (zb::kFinalize | zb::kFlip) : 0);
     a.trigger_late = k == nb - 1;  // followed by the repair check, not by another bucket
+    // the first bucket waits for its predecessor at its start, so it may be a programmatic
+    // dependent of it: after the repair check of a previous step (which triggers at once) its
+    // launch latency is hidden; after any other kernel it starts when that kernel completes
+    a.wait_first = k == 0;
     if (tma) {
       ta.lo = a.lo;
       ta.hi = a.hi;

@@ -368,6 +368,8 @@ struct FusedArgs {
   int nrep;     // bf16 outputs per element: the Nd replicas (ZeRO-1/2), or 1 (a ZeRO-3 layer's shard)
   int chunked;  // 1: CTAs take chunks of kChunkVecs vectors from hdr->chunk (needs mode != 0)
   int trigger_late;  // 1: a dependent launch may start only once this CTA's main loop is done
+  int wait_first;    // 1: launched as a programmatic dependent of whatever precedes it on the
+                     // stream (the first launch of a step); waits for it before anything else
   // ZeRO-3 layer with its gather (kernel variant G): gsrc is the layer's bf16 weights before the
   // update (the concatenated shards, the same memory as reps[0]); each element's old word is
   // copied to the Nd gathered-layer buffers gout[r] before the new weight overwrites it
@@ -427,6 +429,7 @@ template <int DT, int CH, bool G = false>
 __global__ void __launch_bounds__(kThreads, (CH <= 1 && !G) ? 4 : CH <= 4 ? 3 : 2) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   constexpr int BT = kThreads;
   constexpr bool EARLY = CH != 2 || G;
+  if (a.wait_first) pdl_wait();  // the predecessor has completed and its memory is visible
   __shared__ Bias s_bias;
   __shared__ float s_inv;
   __shared__ int s_live;
@@ -789,10 +792,14 @@ struct CastArgs {
 };
 
 // The overflow repair after a fused step may be launched as a programmatic dependent of the last
-// fused launch: it waits for that grid (its header and replica writes) before anything else.
+// fused launch: it waits for that grid (its header and replica writes) before anything else.  It
+// then lets its own dependents launch at once: the only launches that follow it as programmatic
+// dependents are the first fused launch of a next step, which waits at its start, so their
+// launch overlaps this kernel without reading or writing anything before it has completed.
 __global__ void __launch_bounds__(kThreads) cast_allgather_kernel(const __grid_constant__ CastArgs a) {
   __shared__ int s_run, s_live;
   pdl_wait();
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     int run = 1, live = 0;
     if (a.gate == kGateNoOverflow) run = !__ldcg(&a.hdr->pending_flag);
