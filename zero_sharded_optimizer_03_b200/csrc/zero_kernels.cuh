@@ -394,9 +394,9 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 constexpr int kChunkIters = 4;
 constexpr int64_t kChunkVecs = (int64_t)kChunkIters * kThreads;
 
-// CH: gradient replicas loaded per batch (1, 2, 4 or 8).  Built for 3 resident CTAs per SM (24
-// warps) when CH <= 4 and 2 (16 warps, <= 128 registers) when CH = 8: more loads in flight at
-// small fan-in, where each element carries few bytes.
+// CH: gradient replicas loaded per batch (1, 2, 4 or 8).  Small batches leave registers for more
+// resident warps (the budgets are below), so more loads are in flight at small fan-in, where each
+// element carries few bytes.
 //
 // Work distribution: a grid-stride loop over one wave of resident CTAs (every SM owns a fixed
 // share of the window), or, with a.chunked, chunks of kChunkVecs vectors handed out by an atomic
@@ -408,7 +408,9 @@ constexpr int64_t kChunkVecs = (int64_t)kChunkIters * kThreads;
 // Consecutive buckets of one step may be launched as programmatic dependents (fixed split
 // only): the next bucket's CTAs start streaming while this one's last CTAs finish.  The header
 // fields read at the start (t, live, loss scale) change only when a step ends, and a dependent
-// grid waits for its predecessor before it touches the partials and the counters.
+// grid waits for its predecessor before it touches the partials and the counters.  The first
+// launch of a step (wait_first) is a programmatic dependent of whatever precedes it and waits for
+// it before its first instruction, so only its launch overlaps the predecessor.
 //
 // G (ZeRO-3 layer with its gather): every element j of the layer is also the layer's gathered
 // weight j (the gather concatenates the Nd shards, which lie back to back), so one pass reads
