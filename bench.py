@@ -373,6 +373,19 @@ def run_offload(args, w, world, rank, dist, dev, config):
 
 # ----------------------------------------------------------------------------- real ranks
 
+def dist_roofline(S: int, world: int, hbm_gbs: float, link_gbs: float):
+    """Per-rank bytes and ideal time of the real-rank fused step for a shard of S elements over
+    `world` GPUs: HBM carries the rank's own gradient and weight replica windows and its fp32
+    state (2 + 24 + 2 bytes per element); NVLink carries the peers' gradients in and the new
+    weights out to the peers (2 + 2 bytes per element per peer).  Returns (hbm_bytes,
+    link_bytes, bound, ideal_seconds): the slower of the two is the bound."""
+    hbm_bytes = S * (2 + 24 + 2)
+    link_bytes = S * 2 * (world - 1) * 2
+    t_hbm = hbm_bytes / (hbm_gbs * 1e9)
+    t_link = link_bytes / (link_gbs * 1e9)
+    return hbm_bytes, link_bytes, ("nvlink" if t_link > t_hbm else "hbm"), max(t_hbm, t_link)
+
+
 def run_dist(args, w, config):
     """Data parallelism over real GPUs (one process per GPU, torchrun): rank r owns shard r of
     the workload's N parameters and runs the fused kernel over peer memory (symmetric memory);
@@ -457,15 +470,9 @@ def run_dist(args, w, config):
         e2e = {"value": N / (e_ms / args.e2e_steps / 1e3), "unit": "params/s",
                "h2d_bytes_per_step": 2 * N * world, "d2h_bytes_per_step": (2 * N + 112) * world,
                "steps": args.e2e_steps, "result": "every rank's bf16 weight replica + step record"}
-    S = dz.S
-    hbm_bytes = S * (2 + 24 + 2)                   # own gradient, state, own replica (per rank)
-    link_bytes = S * 2 * (world - 1) * 2           # peers' gradients in + weights out
     hbm_peak, hbm_src = peaks()
     link_peak, link_src = nvlink_peak()
-    t_hbm = hbm_bytes / (hbm_peak * 1e9)
-    t_link = link_bytes / (link_peak * 1e9)
-    bound = "nvlink" if t_link > t_hbm else "hbm"
-    ideal = max(t_hbm, t_link)
+    hbm_bytes, link_bytes, bound, ideal = dist_roofline(dz.S, world, hbm_peak, link_peak)
     if rank == 0:
         config.update({"Nd": world, "path": "real ranks: fused kernel over peer memory + NCCL "
                        "step totals", "kernel": "fused_step_kernel (peer loads/stores)",
