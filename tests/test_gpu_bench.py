@@ -39,3 +39,30 @@ def test_bench_line_on_the_short_workload():
     assert c["single_core"]["cores"] == 1 and c["single_core"]["value"] > 0
     assert d["gpu_launches"] == 2 * 40  # fused pass + overflow-repair check per step
     assert d["clocks"] is None or d["clocks"]["sm_mhz"] > 0
+
+
+@pytest.mark.gpu
+def test_bench_real_rank_line_one_rank():
+    """`bench.py --dist` under torchrun, one rank on one GPU (the real-rank path the bench takes
+    on N GPUs): one JSON line, strong scaling, the rank's HBM bytes and no NVLink bytes."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    env = dict(os.environ, NCCL_NVLS_ENABLE="0", TORCH_SYMM_MEM_DISABLE_MULTICAST="1")
+    cmd = ["timeout", "-k", "30", "600", sys.executable, "-m", "torch.distributed.run",
+           "--nnodes", "1", "--nproc-per-node", "1", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.join(ROOT, "bench.py"), "--dist", "--workload",
+           "zero1-gpt2-small", "--steps", "20", "--warmup", "5"]
+    p = subprocess.run(cmd, capture_output=True, text=True, cwd=ROOT, env=env)
+    assert p.returncode == 0, p.stderr[-3000:]
+    lines = [x for x in p.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    N = 124_439_808
+    assert d["scaling"] == "strong" and d["n_gpus"] == 1 and d["config"]["Nd"] == 1
+    assert abs(d["value"] - N / (d["ms_per_step"] / 1e3)) <= 1e-6 * d["value"]
+    r = d["roofline"]
+    assert r["bound"] == "hbm" and r["nvlink_bytes_per_rank"] == 0
+    assert r["hbm_bytes_per_rank"] == 28 * N and 0 < r["frac"] < 1.2
+    assert d["e2e"]["h2d_bytes_per_step"] == 2 * N and d["e2e"]["value"] > 0
