@@ -38,7 +38,7 @@ def test_dist_zero_matches_oracle_one_rank_per_gpu():
 
 # ----------------------------------------------------------------------------- rank windows
 
-def _run_windows(Nd, N, gdt, steps=3, inject=(2, 0, 7)):
+def _run_windows(Nd, N, gdt, steps=3, inject=(2, 0, 7), dynamic=False):
     """Nd data-parallel ranks emulated in one process on one GPU, each with its own buffers laid
     out as dist.DistZero lays them out (full gradient and weight replicas, an S-element state
     shard rebased to global indices, its own workspace).  A step is every rank's
@@ -87,6 +87,8 @@ def _run_windows(Nd, N, gdt, steps=3, inject=(2, 0, 7)):
             st.exp_avg_sq[k] = bases["exp_avg_sq"][k]
         st.workspace = ws.data_ptr()
         zero.zero_workspace_init(ws.data_ptr(), 0, s)
+        if dynamic:  # every rank keeps the same scaler, driven by the combined overflow flag
+            zero.zero_loss_scaler_init(ws.data_ptr(), 1024.0, 2.0, 0.5, 2, s)
         # the initial all-gather: every rank writes bf16 of its shard into every replica
         zero.zero_allgather(bases["master"][0], [p.data_ptr() for p in params], Nd, lo, hi,
                             zero.ZERO_GATE_ALWAYS, None, s)
@@ -96,8 +98,11 @@ def _run_windows(Nd, N, gdt, steps=3, inject=(2, 0, 7)):
     om[:N] = master0
     mm, vm = np.zeros(Np, np.float32), np.zeros(Np, np.float32)
     oreps = [oracle.f32_to_bf16(master0) for _ in range(Nd)]
-    t = 0
+    t, scale, good = 0, 1024.0, 0
+    hpx = dict(hp, dynamic_scale=True, scale_interval=2, scale_growth=2.0, scale_backoff=0.5)
     for k in range(1, steps + 1):
+        if dynamic:  # the gradients carry the scale in force when the step starts
+            sigma = float(np.float32(1e-4 * scale))
         hg = [synth.fill_host(synth.NORMAL, sdt, synth.SEED, synth.grad_stream(k, q), N,
                               sigma=sigma) for q in range(Nd)]
         if k == inject[0] and N > inject[2]:
@@ -117,10 +122,16 @@ def _run_windows(Nd, N, gdt, steps=3, inject=(2, 0, 7)):
         for R in ranks:
             zero.zero_end_step_flip(R["ws"].data_ptr(), s)
             zero.zero_repair_window(Nd, R["lo"], R["hi"], R["st"], s)
-        t, ovf, ss = oracle.zero12_step(Nd, N, 0, odt, hg, om, mm, vm, oreps, hp, t)
+        if dynamic:
+            t, ovf, ss, scale, good = oracle.zero12_step_ex(Nd, N, 0, odt, hg, om, mm, vm, oreps,
+                                                            hpx, t, scale, good)
+        else:
+            t, ovf, ss = oracle.zero12_step(Nd, N, 0, odt, hg, om, mm, vm, oreps, hp, t)
         for R in ranks:
             res = zero.zero_read_result(R["ws"].data_ptr(), s)
             assert (res["overflow"], res["step"]) == (ovf, t), (k, res)
+            if dynamic:
+                assert (res["loss_scale"], res["good_steps"]) == (scale, good), (k, res)
             if not ovf:
                 assert abs(res["grad_sumsq"] - ss) <= 1e-5 * ss
     torch.cuda.synchronize()
@@ -151,3 +162,12 @@ def test_rank_windows_emulated_in_one_process_match_oracle(Nd, N, gdt):
         assert ranks[1]["lo"] == 500_002 and ranks[1]["lo"] % 8 != 0
     if (Nd, N) == (4, 5):
         assert ranks[3]["lo"] == ranks[3]["hi"] == 5
+
+
+@pytest.mark.gpu
+def test_rank_windows_with_dynamic_loss_scale_match_oracle():
+    """The window path with the dynamic loss scaler: fp16 gradients carry each step's scale,
+    every rank's workspace keeps a scaler, and the combined overflow flag (an inf in rank 0's
+    gradient on step 2) backs it off on every rank alike; two clean steps grow it.  Five steps
+    over 3 ranks, every element and every rank's scale sequence equal the oracle's."""
+    _run_windows(3, 100_003, 1, steps=5, dynamic=True)
