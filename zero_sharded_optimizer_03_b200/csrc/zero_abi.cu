@@ -4,6 +4,7 @@
 // the GPU, and enqueues the kernels of zero_kernels.cuh on the caller's stream.  It never
 // allocates memory and never synchronizes except in zero_read_result.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdarg>
@@ -172,6 +173,15 @@ int gather_tma_per_sm() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
   return g_dev[dev].gather_tma_per_sm > 0 ? g_dev[dev].gather_tma_per_sm : 1;
 }
+
+// An NVTX range over a scope (host timeline of a profiler: one range per step, per ZeRO-3
+// layer, per offload chunk).  Without a profiler attached the calls return at once.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
@@ -506,6 +516,7 @@ static int zero3_fused_layers(int Nd, int64_t N, int64_t bucket, const zero_stat
   prof_mark(true, s);
   int64_t off = 0;
   for (int64_t l = 0; l < nl; ++l) {
+    NvtxRange layer_range("zero3 layer: gather + fused update");
     const int64_t Ll = (l + 1) * L <= N ? L : N - l * L;
     const int64_t Sl = (Ll + Nd - 1) / Nd;
     const uint16_t* shards[ZERO_MAX_ND];
@@ -766,6 +777,8 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   if (st->grad_dtype != ZERO_BF16 && st->grad_dtype != ZERO_FP16)
     return fail(ZERO_EINVAL, "grad_dtype=%d", st->grad_dtype);
   if (!st->workspace) return fail(ZERO_EINVAL, "workspace is NULL");
+  static const char* const kStepNames[4] = {"", "zero_step stage 1", "zero_step stage 2", "zero_step stage 3"};
+  NvtxRange range(kStepNames[stage]);
   cudaStream_t s = (cudaStream_t)stream;
   const zb::Consts c = make_consts(hp, Nd);
   void* ws = st->workspace;
@@ -789,6 +802,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     prof_mark(true, s);
     int64_t off = 0;
     for (int64_t l = 0; l < nl; ++l) {  // forward gathers + backward reduce-scatters, layer by layer
+      NvtxRange layer_range("zero3 layer: gather + reduce-scatter");
       const int64_t Ll = (l + 1) * L <= N ? L : N - l * L;
       const int64_t Sl = (Ll + Nd - 1) / Nd;
       const uint16_t* shards[ZERO_MAX_ND];
@@ -1225,6 +1239,7 @@ extern "C" int zero_offload_step(int Nd, int64_t N, int64_t chunk, const zero_of
   if (!st->workspace) return fail(ZERO_EINVAL, "workspace is NULL");
   cudaStream_t s = (cudaStream_t)stream;
   void* ws = st->workspace;
+  NvtxRange range("zero_offload_step");
   if (N == 0) return launch_ws(ws, zb::kWsEnd, 0, s);
   if (!st->grad_dev || !st->param_dev || !st->grad_host || !st->param_host || !st->master_host ||
       !st->exp_avg_host || !st->exp_avg_sq_host)
@@ -1283,6 +1298,7 @@ extern "C" int zero_offload_step(int Nd, int64_t N, int64_t chunk, const zero_of
     for (int64_t k = 0; k < nc; ++k) {
       const int64_t lo = k * C, len = (k + 1) * C < N ? C : N - lo;
       if ((e = cudaEventSynchronize(ring.ev[k])) != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+      NvtxRange chunk_range("host AdamW chunk");
       zh::adam_host(st->master_host + lo, st->exp_avg_host + lo, st->exp_avg_sq_host + lo, st->grad_host + lo,
                     st->param_host + lo, len, hp, h.t + 1, coef, st->host_threads);
       e = cudaMemcpyAsync(st->param_dev + lo, st->param_host + lo, (size_t)len * 2, cudaMemcpyHostToDevice, up);
