@@ -96,6 +96,7 @@ def bytes_per_param(w, two_pass=False, g16=False, fused_layers=False) -> int:
 
 
 L2_BYTES = 126e6  # B200 L2 capacity
+SELF_REPAIR_MAX = 1 << 21  # longest step zero_step runs without an overflow-repair launch
 
 # NVLink figures for the real-rank roofline: a peer copy measured on this machine's B200s (per
 # direction per GPU) and NVIDIA's nominal link rate, used when MEASURED_PEAKS.json has none.
@@ -716,6 +717,8 @@ def main():
         launches_per_step = 3 * nb  # per layer: gather, reduce-scatter, Adam
     elif args.two_pass:
         launches_per_step = 2 * nb  # per bucket: reduce-scatter, Adam + all-gather
+    elif nb == 1 and not tma_path and N <= SELF_REPAIR_MAX:
+        launches_per_step = 1  # the fused kernel repairs a short step itself after a skip
     else:
         launches_per_step = nb + 1  # fused kernel per bucket + the overflow-repair check
 

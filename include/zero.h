@@ -267,7 +267,10 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
  *     overflow-repair check after the last, are programmatic dependent launches on `stream`
  *     (each may start while the previous kernel of the step finishes; it waits for that kernel
  *     before using its results), so nothing else should be enqueued between them: one
- *     zero_step call enqueues the whole step.  The first launch of the register-pipelined pass
+ *     zero_step call enqueues the whole step.  An unbucketed register-pipelined step of at most
+ *     2^21 elements has no repair launch: after an overflow the pass's last CTA rewrites the
+ *     replicas itself (slower for that skipped step, one launch fewer for every other).  The
+ *     first launch of the register-pipelined pass
  *     is a programmatic dependent of whatever precedes it on `stream` and waits for it to
  *     complete before it reads or writes anything, so stream order is kept; after a previous
  *     step's repair check its launch overlaps that kernel.

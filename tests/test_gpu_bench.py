@@ -37,7 +37,7 @@ def test_bench_line_on_the_short_workload():
     c = d["cpu_baseline"]
     assert c["kind"] == "oracle" and c["cores"] >= 1 and c["value"] > 0 and c["sample"]
     assert c["single_core"]["cores"] == 1 and c["single_core"]["value"] > 0
-    assert d["gpu_launches"] == 2 * 40  # fused pass + overflow-repair check per step
+    assert d["gpu_launches"] == 40  # one fused pass per step (it repairs itself after a skip)
     assert d["clocks"] is None or d["clocks"]["sm_mhz"] > 0
 
 

@@ -129,6 +129,10 @@ constexpr int kWavesAdam = 8;
 constexpr int kWavesGather = 16;
 constexpr int kWavesGatherTma = 32;
 
+// Longest unbucketed register-path step whose overflow repair the fused kernel's last CTA does
+// itself (zero_step); longer steps keep the repair launch, whose full grid repairs fast.
+constexpr int64_t kSelfRepairMax = int64_t(1) << 21;
+
 // Fused kernel over a long window: chunks handed out by the workspace counter, or the fixed
 // grid-stride split.  Same-box sweeps at 2^25-2^28 elements, chunks against the best fixed grid:
 // +15% at Nd = 1, +7% at Nd = 4 and, with batches of 4 replicas, +1.4% (124M) to +3.7% (2^28)
@@ -968,6 +972,11 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   // at Nd = 8 the two are equal.  Windows under 2^24 elements keep the register kernel.
   const bool tma_auto = Nd >= 16 && B >= (int64_t(1) << 24);
   const bool tma = al && !(st->flags & ZERO_NO_TMA) && ((st->flags & ZERO_FORCE_TMA) || tma_auto);
+  // A short unbucketed step skips the separate overflow-repair launch: after an overflow the
+  // fused kernel's last CTA rewrites the replicas alone.  On such a step that launch is a large
+  // part of the time (1M elements at Nd = 4: 16.75 -> 15.64 us per step), while a skipped step
+  // becomes slower (one CTA moves the window's 4 + 2Nd bytes per element); skips are rare.
+  const bool self_repair = !tma && nb == 1 && N <= kSelfRepairMax;
   zb::TmaArgs ta;
   if (tma) {
     std::memset(&ta, 0, sizeof ta);
@@ -995,6 +1004,8 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     // dependent of it: after the repair check of a previous step (which triggers at once) its
     // launch latency is hidden; after any other kernel it starts when that kernel completes
     a.wait_first = k == 0;
+    a.self_repair = self_repair;
+    if (self_repair) a.trigger_late = 1;  // the next step may launch once the main loops are done
     if (tma) {
       ta.lo = a.lo;
       ta.hi = a.hi;
@@ -1004,6 +1015,10 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
     } else if ((rc = launch_fused(st->grad_dtype, a, s, k > 0))) {
       return rc;
     }
+  }
+  if (self_repair) {  // the fused kernel's last CTA repairs after a skip: no repair launch
+    prof_mark(false, s);
+    return ZERO_OK;
   }
   // overflow repair: rewrite the replicas from the unchanged state (runs only after a skip);
   // launched as a programmatic dependent of the last fused launch, inside the traced span

@@ -286,8 +286,8 @@ __device__ __forceinline__ double warp_sum(double x) {
 // in CTA order and applies `mode` to the header.  No CTA waits for another (the last one to
 // arrive does the work), so there is no spin and no co-residency assumption.
 template <int NW = kWarps>
-__device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Partial* part, int mode) {
-  if (mode == 0) return;
+__device__ __forceinline__ int block_finish(double sq, int bad, Header* hdr, Partial* part, int mode) {
+  if (mode == 0) return 0;
   __shared__ double r_sq[NW];
   __shared__ int r_bad[NW];
   __shared__ int am_last;
@@ -313,7 +313,7 @@ __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Pa
     am_last = (prev == gridDim.x - 1);
   }
   __syncthreads();
-  if (!am_last) return;
+  if (!am_last) return 0;
   __threadfence();
   double s = 0.0;
   int f = 0;
@@ -343,11 +343,17 @@ __device__ __forceinline__ void block_finish(double sq, int bad, Header* hdr, Pa
       hdr->pending_flag |= fl;
       hdr->pending_sumsq = __dadd_rn(hdr->pending_sumsq, tot);
     }
-    if (mode & kFinalize) end_step(hdr, mode & kFlip);
+    int skipped = 0;
+    if (mode & kFinalize) {
+      end_step(hdr, mode & kFlip);
+      skipped = hdr->last_flag;
+    }
     hdr->done = 0u;
     hdr->chunk = 0ull;  // every CTA has left its chunk loop: ready for the next launch
     __threadfence();
+    return skipped;
   }
+  return 0;
 }
 
 // ------------------------------------------------------------------ K1: fused RS + Adam + AG
@@ -370,6 +376,8 @@ struct FusedArgs {
   int trigger_late;  // 1: a dependent launch may start only once this CTA's main loop is done
   int wait_first;    // 1: launched as a programmatic dependent of whatever precedes it on the
                      // stream (the first launch of a step); waits for it before anything else
+  int self_repair;   // 1: (a step's only launch) after an overflowed step the last CTA rewrites
+                     // the window of every replica from the unchanged state itself
   // ZeRO-3 layer with its gather (kernel variant G): gsrc is the layer's bf16 weights before the
   // update (the concatenated shards, the same memory as reps[0]); each element's old word is
   // copied to the Nd gathered-layer buffers gout[r] before the new weight overwrites it
@@ -436,6 +444,7 @@ __global__ void __launch_bounds__(kThreads, (CH <= 1 && !G) ? 4 : CH <= 4 ? 3 : 
   __shared__ float s_inv;
   __shared__ int s_live;
   __shared__ long long s_chunk;
+  __shared__ int s_repair;
   int live;
   if constexpr (EARLY) {
     live = __ldcg(&a.hdr->live) & 1;
@@ -616,7 +625,29 @@ __global__ void __launch_bounds__(kThreads, (CH <= 1 && !G) ? 4 : CH <= 4 ? 3 : 
     for (int r = 0; r < a.nrep; ++r) a.reps[r][i] = w;
   }
   pdl_wait();  // a programmatic dependent: the previous bucket has completed
-  block_finish<BT / 32>(sq, bad, a.hdr, a.part, a.mode);
+  const int skipped = block_finish<BT / 32>(sq, bad, a.hdr, a.part, a.mode);
+  // short window: the last CTA to finish repairs the replicas after a skip.  Every other CTA has
+  // published its speculative stores (fence, then its arrival) before the last one arrived, so
+  // these stores come after them.
+  if (a.self_repair) {
+    __syncthreads();
+    if (threadIdx.x == 0) s_repair = skipped;
+    __syncthreads();
+    if (s_repair) {
+      for (int64_t j = threadIdx.x; j < sp8.nvec; j += BT) {
+        const int64_t i = sp8.vlo + (j << 3);
+        float P[8];
+        unpack(ld_stream(sp + i), ld_stream(sp + i + 4), P);
+        const uint4 w = pack_bf16x8(P);
+        for (int r = 0; r < a.nrep; ++r) st_stream(a.reps[r] + i, w);
+      }
+      for (int64_t e = threadIdx.x; e < sp8.nrest; e += BT) {
+        const int64_t i = sp8.scalar_index(a.lo, e);
+        const uint16_t w = to_bf16(sp[i]);
+        for (int r = 0; r < a.nrep; ++r) a.reps[r][i] = w;
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------ K3: RS into an fp32 shard
