@@ -367,7 +367,9 @@ int zero_test_inject_stall(int64_t unit);
  * first element).  finalize = 0 leaves the step open: the caller combines the pending
  * overflow flag (MAX) and sum of squares (SUM) of every rank in the workspace header (int32 at
  * byte 4, double at byte 8), then calls zero_end_step_flip and zero_repair_window; finalize != 0
- * ends the step here (single GPU).  No clipping (it needs the global norm first).  Async. */
+ * ends the step here (single GPU) and, after an overflow, rewrites the window of every replica
+ * from the unchanged state (a repair check launched after the pass).  No clipping (it needs the
+ * global norm first).  Async. */
 int zero_fused_window(int Nd, int64_t lo, int64_t hi, const zero_state_t *st,
                       const zero_hparams_t *hp, int finalize, void *stream);
 

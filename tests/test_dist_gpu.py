@@ -171,3 +171,48 @@ def test_rank_windows_with_dynamic_loss_scale_match_oracle():
     gradient on step 2) backs it off on every rank alike; two clean steps grow it.  Five steps
     over 3 ranks, every element and every rank's scale sequence equal the oracle's."""
     _run_windows(3, 100_003, 1, steps=5, dynamic=True)
+
+
+@pytest.mark.gpu
+def test_single_finalized_window_matches_oracle_and_repairs():
+    """zero_fused_window with finalize over the whole vector (one GPU, the step ended by the
+    pass itself): three steps with an overflow on step 2; after the skip every replica is
+    rewritten from the unchanged state, and every element equals the oracle's."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import synth
+    import zero_sharded_optimizer_03_b200 as zero
+    Nd, N = 4, 300_007
+    s = torch.cuda.current_stream().cuda_stream
+    hp = dict(lr=1e-3, weight_decay=0.01, loss_scale=1.0)
+    buf = zero.ZeroBuffers(2, Nd, N)
+    master0 = synth.fill_host(synth.NORMAL, synth.F32, synth.SEED, synth.MASTER_STREAM, N,
+                              sigma=0.02)
+    buf.master[0][:N].copy_(torch.from_numpy(master0))
+    buf.init_workspace(0)
+    buf.sync_params_from_master()
+    S, Np, _ = oracle.partition(N, Nd)
+    om = np.zeros(Np, np.float32)
+    om[:N] = master0
+    mm, vm = np.zeros(Np, np.float32), np.zeros(Np, np.float32)
+    oreps = [oracle.f32_to_bf16(master0) for _ in range(Nd)]
+    t = 0
+    for k in (1, 2, 3):
+        hg = [synth.fill_host(synth.NORMAL, synth.BF16, synth.SEED, synth.grad_stream(k, q), N,
+                              sigma=1e-3) for q in range(Nd)]
+        if k == 2:
+            hg[1][4321] = 0x7F80
+        for q in range(Nd):
+            buf.grads[q].view(torch.int16).copy_(torch.from_numpy(hg[q].view(np.int16)))
+        zero.zero_fused_window(Nd, 0, N, buf.state, zero.hparams(**hp), True, s)
+        t, ovf, ss = oracle.zero12_step(Nd, N, 0, oracle.BF16, hg, om, mm, vm, oreps, hp, t)
+        res = buf.result()
+        assert (res["overflow"], res["step"]) == (ovf, t) == (int(k == 2), (1, 1, 2)[k - 1])
+        for q in range(Nd):  # the replicas hold the committed weights after every step
+            got = buf.params[q].view(torch.int16).cpu().numpy().view(np.uint16)
+            assert got.tobytes() == oreps[q].tobytes(), (k, q)
+    live = buf.live()
+    assert buf.master[live].cpu().numpy().tobytes() == om.tobytes()
+    assert buf.exp_avg_sq[live].cpu().numpy().tobytes() == vm.tobytes()

@@ -1371,9 +1371,24 @@ extern "C" int zero_fused_window(int Nd, int64_t lo, int64_t hi, const zero_stat
   a.lo = lo;
   a.hi = hi;
   a.mode = zb::kAccSet | (finalize ? (zb::kFinalize | zb::kFlip) : 0);
+  a.trigger_late = finalize != 0;  // followed by the repair check
   cudaStream_t s = (cudaStream_t)stream;
   prof_mark(true, s);
   rc = launch_fused(st->grad_dtype, a, s);
+  if (!rc && finalize) {  // the step ended here: after an overflow, rewrite the window's replicas
+    zb::CastArgs r;
+    std::memset(&r, 0, sizeof r);
+    r.src[0] = st->master[0];
+    r.src[1] = st->master[1];
+    for (int q = 0; q < Nd; ++q) r.reps[q] = st->params[q];
+    r.nrep = Nd;
+    r.gate = zb::kGateRepair;
+    r.lo = lo;
+    r.hi = hi;
+    r.hdr = header(st->workspace);
+    r.vec = al;
+    rc = launch_cast(r, s, true);
+  }
   prof_mark(false, s);
   return rc;
 }
