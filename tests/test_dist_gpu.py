@@ -105,7 +105,7 @@ def _run_windows(Nd, N, gdt, steps=3, inject=(2, 0, 7), dynamic=False):
             sigma = float(np.float32(1e-4 * scale))
         hg = [synth.fill_host(synth.NORMAL, sdt, synth.SEED, synth.grad_stream(k, q), N,
                               sigma=sigma) for q in range(Nd)]
-        if k == inject[0] and N > inject[2]:
+        if inject is not None and k == inject[0] and N > inject[2]:
             hg[inject[1]][inject[2]] = inf_bits
         for q in range(Nd):
             grads[q][:N].view(torch.int16).copy_(torch.from_numpy(hg[q].view(np.int16)))
@@ -216,3 +216,29 @@ def test_single_finalized_window_matches_oracle_and_repairs():
     live = buf.live()
     assert buf.master[live].cpu().numpy().tobytes() == om.tobytes()
     assert buf.exp_avg_sq[live].cpu().numpy().tobytes() == vm.tobytes()
+
+
+def _random_window_cases(n_cases=12, seed=2028):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    cases = []
+    for k in range(n_cases):
+        Nd = int(rng.choice([2, 3, 4, 5, 7, 8]))
+        N = int(rng.choice([9, 1001, 65_537, 200_003, 524_291]))
+        gdt = int(rng.choice([0, 1]))
+        dynamic = bool(gdt == 1 and rng.random() < 0.5)
+        rank = int(rng.integers(0, Nd))
+        index = int(rng.integers(0, N))
+        inject = (2, rank, index) if rng.random() < 0.7 else None
+        cases.append((k, Nd, N, gdt, dynamic, inject))
+    return cases
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", _random_window_cases(), ids=lambda c: "case%d" % c[0])
+def test_randomized_rank_windows_against_oracle(case):
+    """Seeded random rank-window cases (Nd, N, gradient dtype, dynamic loss scale, an overflow in
+    a random rank's gradient at a random index or none), four steps each, every element of every
+    rank's shard and replica against the oracle."""
+    k, Nd, N, gdt, dynamic, inject = case
+    _run_windows(Nd, N, gdt, steps=4, inject=inject, dynamic=dynamic)
