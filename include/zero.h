@@ -156,7 +156,8 @@ typedef struct {
     uint16_t *param_shard;  /* stage 3: bf16 weights, the Nd shards of every layer (padded) */
     int64_t grad_layer_stride;
     int64_t param_layer_stride;
-    void *workspace;        /* zero_workspace_bytes() bytes, initialised by zero_workspace_init */
+    void *workspace;        /* zero_workspace_bytes() bytes, 16-byte aligned, initialised by
+                               zero_workspace_init */
 } zero_state_t;
 
 /* Per-GPU model-state memory in GiB (2^30 bytes). */
@@ -177,7 +178,10 @@ const char *zero_version(void);
 int zero_partition(int64_t N, int Nd, zero_partition_t *out);
 
 /* Bytes of device workspace a step needs (a small constant: step counter, overflow flag,
- * sum of squares, per-CTA partials).  One workspace per optimizer (it carries the step count). */
+ * sum of squares, per-CTA partials).  One workspace per optimizer (it carries the step count).
+ * Every call that takes a workspace refuses, with ZERO_EINVAL and before any device work, a
+ * NULL one or one whose address is not a multiple of 16 (the kernels update its doubles and
+ * 64-bit counters in place). */
 size_t zero_workspace_bytes(void);
 
 /* Sets the workspace to "t completed updates, nothing pending, state copy 0 live".  Async. */

@@ -164,6 +164,25 @@ def test_entry_points_validate_before_touching_the_device(zero):
         assert zero.lib.zero_last_error().decode() != ""
 
 
+def test_misaligned_workspace_is_refused(zero):
+    """A workspace off a 16-byte boundary is refused before any device work (the kernels would
+    update its doubles and 64-bit counters at misaligned addresses)."""
+    hp = zero.hparams(1e-3)
+    st = zero.zero_state_t()
+    st.workspace = 4096 + 8  # fake, never dereferenced
+    cases = [
+        lambda: zero.zero_step(2, 4, 10, 0, st, hp),
+        lambda: zero.zero_workspace_init(4096 + 8, 0),
+        lambda: zero.zero_loss_scaler_init(4096 + 4, 1024.0),
+        lambda: zero.zero_allgather(16, [16] * 2, 2, 0, 8, 1, 4096 + 8),
+        lambda: zero.zero_reduce_scatter([16] * 4, 0, 4, 0, 8, hp, 16, 4096 + 8),
+    ]
+    for k, call in enumerate(cases):
+        with pytest.raises(zero.ZeroError) as e:
+            call()
+        assert e.value.code == zero.ZERO_EINVAL and "16-byte aligned" in str(e.value), k
+
+
 def test_fused_step_refuses_clipping(zero):
     st = zero.zero_state_t()
     st.grad_dtype = zero.ZERO_BF16

@@ -35,6 +35,14 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The kernels read and update the workspace's doubles and 64-bit counters in place: a NULL
+// workspace, or one off a 16-byte boundary, is rejected before anything is launched.
+int check_ws(const void* ws) {
+  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (!aligned16(ws)) return fail(ZERO_EINVAL, "workspace %p is not 16-byte aligned", ws);
+  return ZERO_OK;
+}
+
 // Resident CTAs per SM for each kernel, cached per device (occupancy does not change).
 constexpr int kMaxDevices = 64;
 enum KernelId {
@@ -613,13 +621,14 @@ int zero_partition(int64_t N, int Nd, zero_partition_t* out) {
 size_t zero_workspace_bytes(void) { return zb::kWorkspaceBytes; }
 
 int zero_workspace_init(void* ws, int64_t t, void* stream) {
-  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (const int rc = check_ws(ws)) return rc;
   if (t < 0) return fail(ZERO_EINVAL, "t=%lld < 0", (long long)t);
   return launch_ws(ws, zb::kWsInit, t, (cudaStream_t)stream);
 }
 
 int zero_read_result(const void* ws, zero_step_result_t* out, void* stream) {
-  if (!ws || !out) return fail(ZERO_EINVAL, "workspace or out is NULL");
+  if (!out) return fail(ZERO_EINVAL, "out is NULL");
+  if (const int rc = check_ws(ws)) return rc;
   zb::Header h;
   cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof h, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(result)");
@@ -655,7 +664,7 @@ int zero_profile_events(void* start_event, void* stop_event) {
 
 int zero_loss_scaler_init(void* ws, double init_scale, double growth_factor, double backoff_factor,
                           int64_t growth_interval, void* stream) {
-  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (const int rc = check_ws(ws)) return rc;
   if (!(init_scale > 0) || !std::isfinite(init_scale)) return fail(ZERO_EINVAL, "init_scale must be finite and > 0");
   if (!(growth_factor >= 1) || !std::isfinite(growth_factor)) return fail(ZERO_EINVAL, "growth_factor must be >= 1");
   if (!(backoff_factor > 0 && backoff_factor <= 1)) return fail(ZERO_EINVAL, "backoff_factor must be in (0, 1]");
@@ -672,12 +681,12 @@ int zero_test_inject_stall(int64_t unit) {
 }
 
 int zero_begin_step(void* ws, void* stream) {
-  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (const int rc = check_ws(ws)) return rc;
   return launch_ws(ws, zb::kWsBegin, 0, (cudaStream_t)stream);
 }
 
 int zero_end_step(void* ws, void* stream) {
-  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (const int rc = check_ws(ws)) return rc;
   return launch_ws(ws, zb::kWsEnd, 0, (cudaStream_t)stream);
 }
 
@@ -689,7 +698,8 @@ int zero_reduce_scatter(const uint16_t* const* grads, int dtype, int Nd, int64_t
   if ((rc = check_hp(hp))) return rc;
   if (dtype != ZERO_BF16 && dtype != ZERO_FP16) return fail(ZERO_EINVAL, "dtype=%d", dtype);
   if (lo == hi) return ZERO_OK;  // empty window: nothing to reduce or to report
-  if (!grad_out || !ws) return fail(ZERO_EINVAL, "grad_out or workspace is NULL");
+  if (!grad_out) return fail(ZERO_EINVAL, "grad_out is NULL");
+  if ((rc = check_ws(ws))) return rc;
   zb::RsArgs a;
   std::memset(&a, 0, sizeof a);
   bool al = aligned16(grad_out);
@@ -715,8 +725,9 @@ int zero_adam_shard(float* master, float* exp_avg, float* exp_avg_sq, const floa
   if (rc) return rc;
   if ((rc = check_hp(hp))) return rc;
   if (lo == hi) return ZERO_OK;
-  if (!master || !exp_avg || !exp_avg_sq || !grad || !ws)
-    return fail(ZERO_EINVAL, "master, exp_avg, exp_avg_sq, grad and workspace must be non-NULL");
+  if (!master || !exp_avg || !exp_avg_sq || !grad)
+    return fail(ZERO_EINVAL, "master, exp_avg, exp_avg_sq and grad must be non-NULL");
+  if ((rc = check_ws(ws))) return rc;
   zb::AdamArgs a;
   std::memset(&a, 0, sizeof a);
   a.p[0] = a.p[1] = master;
@@ -743,7 +754,7 @@ int zero_allgather(const float* master, uint16_t* const* replicas, int Nd, int64
   if (rc) return rc;
   if ((rc = check_window(lo, hi))) return rc;
   if (gate != ZERO_GATE_ALWAYS && gate != ZERO_GATE_NO_OVERFLOW) return fail(ZERO_EINVAL, "gate=%d", gate);
-  if (gate == ZERO_GATE_NO_OVERFLOW && !ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (gate == ZERO_GATE_NO_OVERFLOW && (rc = check_ws(ws))) return rc;
   if (lo == hi) return ZERO_OK;
   if (!master) return fail(ZERO_EINVAL, "master is NULL");
   zb::CastArgs a;
@@ -780,7 +791,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   if (N < 0 || bucket < 0) return fail(ZERO_EINVAL, "N and bucket must be >= 0");
   if (st->grad_dtype != ZERO_BF16 && st->grad_dtype != ZERO_FP16)
     return fail(ZERO_EINVAL, "grad_dtype=%d", st->grad_dtype);
-  if (!st->workspace) return fail(ZERO_EINVAL, "workspace is NULL");
+  if ((rc = check_ws(st->workspace))) return rc;
   static const char* const kStepNames[4] = {"", "zero_step stage 1", "zero_step stage 2", "zero_step stage 3"};
   NvtxRange range(kStepNames[stage]);
   cudaStream_t s = (cudaStream_t)stream;
@@ -1251,7 +1262,7 @@ extern "C" int zero_offload_step(int Nd, int64_t N, int64_t chunk, const zero_of
   if (!st) return fail(ZERO_EINVAL, "state is NULL");
   if (N < 0 || chunk < 0) return fail(ZERO_EINVAL, "N and chunk must be >= 0");
   if (st->grad_dtype != ZERO_BF16 && st->grad_dtype != ZERO_FP16) return fail(ZERO_EINVAL, "grad_dtype=%d", st->grad_dtype);
-  if (!st->workspace) return fail(ZERO_EINVAL, "workspace is NULL");
+  if ((rc = check_ws(st->workspace))) return rc;
   cudaStream_t s = (cudaStream_t)stream;
   void* ws = st->workspace;
   NvtxRange range("zero_offload_step");
@@ -1342,7 +1353,8 @@ extern "C" int zero_fused_window(int Nd, int64_t lo, int64_t hi, const zero_stat
   if (rc) return rc;
   if ((rc = check_window(lo, hi))) return rc;
   if ((rc = check_hp(hp))) return rc;
-  if (!st || !st->workspace) return fail(ZERO_EINVAL, "state or workspace is NULL");
+  if (!st) return fail(ZERO_EINVAL, "state is NULL");
+  if ((rc = check_ws(st->workspace))) return rc;
   if (st->grad_dtype != ZERO_BF16 && st->grad_dtype != ZERO_FP16) return fail(ZERO_EINVAL, "grad_dtype=%d", st->grad_dtype);
   if (hp->max_grad_norm > 0) return fail(ZERO_EINVAL, "the fused pass cannot clip (needs the global norm first)");
   bool al = true;
@@ -1394,7 +1406,7 @@ extern "C" int zero_fused_window(int Nd, int64_t lo, int64_t hi, const zero_stat
 }
 
 extern "C" int zero_end_step_flip(void* ws, void* stream) {
-  if (!ws) return fail(ZERO_EINVAL, "workspace is NULL");
+  if (const int rc = check_ws(ws)) return rc;
   return launch_ws(ws, zb::kWsEndFlip, 0, (cudaStream_t)stream);
 }
 
@@ -1403,6 +1415,7 @@ extern "C" int zero_repair_window(int Nd, int64_t lo, int64_t hi, const zero_sta
   if (rc) return rc;
   if ((rc = check_window(lo, hi))) return rc;
   if (!st || !st->workspace || !st->master[0] || !st->master[1]) return fail(ZERO_EINVAL, "state is incomplete");
+  if ((rc = check_ws(st->workspace))) return rc;
   if (lo == hi) return ZERO_OK;
   bool al = aligned16(st->master[0]) && aligned16(st->master[1]);
   if ((rc = check_ptrs(st->params, Nd, "params", &al))) return rc;
