@@ -98,8 +98,9 @@ def bytes_per_param(w, two_pass=False, g16=False, fused_layers=False) -> int:
 L2_BYTES = 126e6  # B200 L2 capacity
 SELF_REPAIR_MAX = 1 << 21  # longest step zero_step runs without an overflow-repair launch
 
-# NVLink figures for the real-rank roofline: a peer copy measured on this machine's B200s (per
-# direction per GPU) and NVIDIA's nominal link rate, used when MEASURED_PEAKS.json has none.
+# NVLink figures for the real-rank roofline: a peer copy measured between B200s of an NVSwitch
+# node (per direction per GPU) and NVIDIA's nominal link rate, used when MEASURED_PEAKS.json has
+# none.
 NVLINK_PEER_COPY_GBS = 770.0
 NVLINK_NOMINAL_GBS = 900.0
 
@@ -114,14 +115,14 @@ def peaks():
 
 def nvlink_peak():
     """(GB/s per direction per GPU, source) for NVLink: MEASURED_PEAKS.json if it has a figure,
-    else the machine's measured peer copy."""
+    else the measured B200 peer copy."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
         for key in ("nvlink_gbs", "nvlink_peer_gbs", "p2p_gbs"):
             if key in d:
                 return float(d[key]), "measured (MEASURED_PEAKS.json %s)" % key
-    return NVLINK_PEER_COPY_GBS, ("peer copy measured on this pool, per direction (nominal %g)"
+    return NVLINK_PEER_COPY_GBS, ("measured B200 peer copy, per direction (nominal %g)"
                                   % NVLINK_NOMINAL_GBS)
 
 

@@ -128,7 +128,7 @@ def test_short_workloads_cycle_optimizer_instances():
 def test_real_rank_roofline_bytes_and_bound():
     """The real-rank step's roofline: one GPU moves only its HBM bytes; with peers each element
     of a rank's shard crosses NVLink once per peer in (gradient) and once out (weights), so at
-    the pool's 770 GB/s peer copy against ~6.5 TB/s of HBM the step is NVLink-bound from 2 GPUs."""
+    the measured 770 GB/s B200 peer copy against ~6.5 TB/s of HBM the step is NVLink-bound from 2 GPUs."""
     S = 1 << 25
     hbm, link, bound, ideal = bench.dist_roofline(S, 1, 6527.8, 770.0)
     assert (hbm, link, bound) == (28 * S, 0, "hbm") and ideal == 28 * S / 6527.8e9

@@ -976,7 +976,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
   a.Nd = Nd;
   a.nrep = Nd;
   a.vec = al;
-  // The TMA pipeline wins where many loads must be in flight per element (same box, with its
+  // The TMA pipeline wins where many loads must be in flight per element (one B200, with its
   // multi-wave grid: Nd = 64, 2^28: 6671 GB/s against 6091 for the register kernel; Nd = 16,
   // 1.3e9 in one bucket: 6635 against 6229; in 52 buckets of 25M, with the buckets launched as
   // programmatic dependents, which hides the TMA kernel's per-launch set-up: 6555 against 6115);
