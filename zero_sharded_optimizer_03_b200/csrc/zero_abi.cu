@@ -543,6 +543,7 @@ static int zero3_fused_layers(int Nd, int64_t N, int64_t bucket, const zero_stat
     if (tma_gather && (rc = do_gather_tma(shards, Nd, Ll, outs, Nd, ws, s))) return rc;
     zb::FusedArgs a;
     std::memset(&a, 0, sizeof a);
+    a.prefetch = 1;  // the step's own buffers: this GPU's memory
     bool fal = true;
     for (int r = 0; r < Nd; ++r) {
       a.grads[r] = st->grads[r] + l * st->grad_layer_stride;
@@ -960,6 +961,7 @@ int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t* 
       return fail(ZERO_EINVAL, "ZERO_FUSED needs both state copies (master/exp_avg/exp_avg_sq [0] and [1])");
   zb::FusedArgs a;
   std::memset(&a, 0, sizeof a);
+  a.prefetch = 1;  // the step's own buffers: this GPU's memory
   for (int r = 0; r < Nd; ++r) {
     a.grads[r] = st->grads[r];
     a.reps[r] = st->params[r];

@@ -417,6 +417,8 @@ struct FusedArgs {
                      // stream (the first launch of a step); waits for it before anything else
   int self_repair;   // 1: (a step's only launch) after an overflowed step the last CTA rewrites
                      // the window of every replica from the unchanged state itself
+  int prefetch;      // 1: a thread's second vector is prefetched to L2 (set only where every
+                     // buffer is this GPU's memory; never for a window that reads peers' memory)
   // ZeRO-3 layer with its gather (kernel variant G): gsrc is the layer's bf16 weights before the
   // update (the concatenated shards, the same memory as reps[0]); each element's old word is
   // copied to the Nd gathered-layer buffers gout[r] before the new weight overwrites it
@@ -607,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, (CH <= 1 && !G) ? 4 : CH <= 4 ? 3 : 
       // A window a little larger than one round of the grid leaves a second vector to some
       // threads; its lines start for L2 now, with the first round's loads, so that its loads
       // after the first update hit L2 (1M elements at Nd = 4: 0.2 us of a 14.7 us step).
-      if (j + stride < sp8.nvec) {
+      if (a.prefetch && j + stride < sp8.nvec) {
         const int64_t i2 = sp8.vlo + ((j + stride) << 3);
         prefetch_l2(sp + i2);
         prefetch_l2(sm + i2);
