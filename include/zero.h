@@ -296,7 +296,10 @@ int zero3_gather_layer(const uint16_t *const *shards, int Nd, int64_t L, uint16_
  *     parameter instead of 36 + 4*Nd, for a second fp32 state copy (12 bytes per parameter);
  *     no grad_shard; refuses max_grad_norm > 0 and ZERO_BF16_GRAD_SHARD (ZERO_EINVAL).
  * Every path skips the whole update (state, weights, t) when any reduced gradient element is
- * inf or NaN.  Asynchronous: call zero_read_result to learn whether the step was skipped. */
+ * inf or NaN.  Every buffer of `st` is memory of the current device (the register-pipelined
+ * pass may prefetch a thread's next vector into L2; a pass over other GPUs' memory is
+ * zero_fused_window, which never prefetches).  Asynchronous: call zero_read_result to learn
+ * whether the step was skipped. */
 int zero_step(int stage, int Nd, int64_t N, int64_t bucket, const zero_state_t *st,
               const zero_hparams_t *hp, void *stream);
 
